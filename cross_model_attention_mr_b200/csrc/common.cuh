@@ -1,0 +1,82 @@
+// Shared device-side definitions for the libmr kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/mr.h"
+
+namespace mr {
+
+// Workspace header shared by every entry point: a status word and work-queue counters.
+struct WsHeader {
+  uint32_t status;         // first device-side error (mr_status), 0 = none
+  uint32_t detail;         // where it happened (kernel-specific code)
+  uint32_t counters[14];   // dynamic work queues (zeroed by the host before each launch)
+};
+static_assert(sizeof(WsHeader) == 64, "header layout");
+constexpr size_t kWsHeaderBytes = 256;
+
+__device__ __forceinline__ void set_status(WsHeader* ws, uint32_t code, uint32_t detail) {
+  if (atomicCAS(&ws->status, 0u, code) == 0u) ws->detail = detail;
+}
+
+// Logit bias b(h, i, j) for a causal pair j <= i: the largest applicable term, 0 if none.
+// (Synthetic stand-in for sink / local-window / retrieval-head structure.)
+struct Bias {
+  int sink_len;
+  float sink_bias;
+  int window;
+  float window_bias;
+  const float* kb;  // [heads][n_kb] or nullptr; -inf = no term
+  int kb_block;
+  int n_kb;
+};
+
+inline Bias make_bias(const mr_logit_bias* b) {
+  Bias r{0, 0.f, 0, 0.f, nullptr, 1, 0};
+  if (b) {
+    r.sink_len = b->sink_len;
+    r.sink_bias = b->sink_bias;
+    r.window = b->window;
+    r.window_bias = b->window_bias;
+    r.kb = b->kb_bias;
+    r.kb_block = b->kb_block > 0 ? b->kb_block : 1;
+    r.n_kb = b->n_kb;
+  }
+  return r;
+}
+
+__device__ __forceinline__ float bias_term(const Bias& b, int h, int i, int j) {
+  float best = -INFINITY;
+  if (j < b.sink_len) best = b.sink_bias;
+  if (i - j < b.window) best = fmaxf(best, b.window_bias);
+  if (b.kb != nullptr) best = fmaxf(best, __ldg(b.kb + (size_t)h * b.n_kb + j / b.kb_block));
+  return best == -INFINITY ? 0.f : best;
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// Rank of key block J among the kept blocks of one row: number of kept blocks below J.
+__device__ __forceinline__ int kept_rank(const uint32_t* bits, int J) {
+  int r = 0;
+  const int w = J >> 5;
+  for (int t = 0; t < w; ++t) r += __popc(bits[t]);
+  const uint32_t below = (J & 31) ? (bits[w] & ((1u << (J & 31)) - 1u)) : 0u;
+  return r + __popc(below);
+}
+
+}  // namespace mr

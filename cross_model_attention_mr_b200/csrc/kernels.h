@@ -1,0 +1,66 @@
+// Host-side launchers of the libmr kernels (internal to the library; not part of the C-ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace mr {
+
+struct CompressArgs {
+  const void* Q;
+  const void* K;
+  mr_dtype dt;
+  int H, L, d, block;
+  float scale, p;
+  Bias bias;
+  WsHeader* ws;
+  float* lse_ws;    // [H][L] natural-log row normaliser (workspace)
+  int* count_ws;    // [H * nqb]
+  mr_bsr map;
+  cudaStream_t stream;
+};
+
+struct RetrieveArgs {
+  mr_bsr map;
+  const float* W;
+  int H_r;
+  const void* V;
+  void* O;
+  mr_dtype dt;
+  int d_v, n_req;
+  const int64_t* v_req_off;
+  int64_t v_req_stride, v_head_stride;
+  WsHeader* ws;
+  cudaStream_t stream;
+};
+
+struct DenseArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  void* O;
+  mr_dtype dt;
+  int H, d, d_v;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  const int32_t* q_offset;
+  int n_seq, total_q, total_k;
+  float scale;
+  Bias bias;
+  WsHeader* ws;
+  cudaStream_t stream;
+};
+
+// SIMT (CUDA-core) kernels: fp32 inputs, and bf16 where no tensor-core kernel applies.
+cudaError_t simt_compress(const CompressArgs& a);
+cudaError_t simt_retrieve(const RetrieveArgs& a);
+cudaError_t simt_dense(const DenseArgs& a);
+
+// Shared by every compress path: exclusive scan of the kept counts into row_ptr, nnz, capacity.
+cudaError_t launch_scan_counts(const int* count, int n, mr_bsr map, WsHeader* ws, cudaStream_t st);
+
+cudaError_t launch_export(const mr_bsr& map, int64_t n_tiles, float* out, cudaStream_t st);
+
+}  // namespace mr

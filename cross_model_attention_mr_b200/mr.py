@@ -1,0 +1,292 @@
+"""Python binding of libmr (argument marshalling only; every step of the path runs in libmr's kernels).
+
+The names follow the C-ABI in ``include/mr.h``: ``compress`` -> ``mr_compress``, ``retrieve`` ->
+``mr_retrieve``, ``dense_ref`` -> ``mr_dense_ref``.  PyTorch is used for device memory and streams.
+Importing this module loads ``libmr.so`` and raises ``ImportError`` if it has not been built:
+there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmr.so")
+
+MR_OK, MR_ERR_INVALID_ARG, MR_ERR_UNSUPPORTED, MR_ERR_CAPACITY = 0, 1, 2, 3
+MR_ERR_CUDA, MR_ERR_TIMEOUT, MR_ERR_DEVICE_CHECK, MR_ERR_RANGE = 4, 5, 6, 7
+MR_BF16, MR_F32 = 0, 1
+
+_c_i32, _c_i64, _c_f32, _c_p, _c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+
+
+class LogitBias(ctypes.Structure):
+    _fields_ = [("sink_len", _c_i32), ("sink_bias", _c_f32), ("window", _c_i32), ("window_bias", _c_f32),
+                ("kb_bias", _c_p), ("kb_block", _c_i32), ("n_kb", _c_i32)]
+
+
+class BSR(ctypes.Structure):
+    _fields_ = [("H_s", _c_i32), ("L", _c_i32), ("block", _c_i32), ("val_dtype", ctypes.c_int),
+                ("capacity_tiles", _c_i64), ("row_ptr", _c_p), ("col_idx", _c_p), ("vals", _c_p),
+                ("kept_mass", _c_p), ("kept_bits", _c_p), ("mass", _c_p), ("lse", _c_p), ("nnz", _c_p)]
+
+
+EXPORTS = {
+    "mr_version": ([], ctypes.c_int),
+    "mr_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "mr_device_supported": ([], ctypes.c_int),
+    "mr_compress_workspace_bytes": ([ctypes.c_int] * 4, _c_sz),
+    "mr_bsr_max_tiles": ([ctypes.c_int] * 3, _c_i64),
+    "mr_compress": ([_c_p, _c_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _c_f32, _c_f32,
+                     ctypes.POINTER(LogitBias), ctypes.POINTER(BSR), _c_p, _c_sz, _c_p], ctypes.c_int),
+    "mr_retrieve_workspace_bytes": ([ctypes.POINTER(BSR), ctypes.c_int, ctypes.c_int, ctypes.c_int], _c_sz),
+    "mr_retrieve": ([ctypes.POINTER(BSR), _c_p, ctypes.c_int, _c_p, _c_p, ctypes.c_int, ctypes.c_int,
+                     ctypes.c_int, _c_p, _c_i64, _c_i64, _c_p, _c_sz, _c_p], ctypes.c_int),
+    "mr_dense_ref_workspace_bytes": ([ctypes.c_int], _c_sz),
+    "mr_dense_ref": ([_c_p, _c_p, _c_p, _c_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                      _c_p, _c_p, _c_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _c_f32,
+                      ctypes.POINTER(LogitBias), _c_p, _c_sz, _c_p], ctypes.c_int),
+    "mr_sync_status": ([_c_p, _c_p], ctypes.c_int),
+    "mr_bsr_nnz": ([ctypes.POINTER(BSR), ctypes.POINTER(_c_i64), _c_p], ctypes.c_int),
+    "mr_bsr_export": ([ctypes.POINTER(BSR), _c_i64, _c_p, _c_p], ctypes.c_int),
+    "mr_profile_enable": ([ctypes.c_int], ctypes.c_int),
+    "mr_profile_read": ([_c_p, _c_p, ctypes.c_int], ctypes.c_int),
+    "mr_kernel_name": ([ctypes.c_int], ctypes.c_char_p),
+    "mr_kernel_launches": ([], _c_i64),
+}
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with __graft_entry__.build()")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (args, res) in EXPORTS.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+LIB = _load()
+
+
+class MRError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {LIB.mr_status_string(code).decode()} (status {code})")
+
+
+def check(code: int, where: str) -> None:
+    if code != MR_OK:
+        raise MRError(code, where)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return MR_BF16
+    if t.dtype == torch.float32:
+        return MR_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _torch_dtype(dt: int):
+    return torch.bfloat16 if dt == MR_BF16 else torch.float32
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+class Workspace:
+    """Device workspace (256-byte aligned torch allocation)."""
+
+    def __init__(self, nbytes: int, device="cuda"):
+        self.nbytes = max(256, int(nbytes))
+        self.buf = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device)
+        off = (-self.buf.data_ptr()) % 256
+        self.ptr = self.buf.data_ptr() + off
+
+    def sync_status(self, stream=None) -> int:
+        return LIB.mr_sync_status(self.ptr, _stream(stream))
+
+
+class Bias:
+    """Device-side logit bias (holds the kb_bias tensor alive)."""
+
+    def __init__(self, sink_len=0, sink_bias=0.0, window=0, window_bias=0.0, kb_bias=None,
+                 kb_block=0, device="cuda"):
+        self.kb = None
+        if kb_bias is not None:
+            kb = torch.as_tensor(np.ascontiguousarray(kb_bias, dtype=np.float32))
+            self.kb = kb.to(device).contiguous()
+        self.c = LogitBias(int(sink_len), float(sink_bias), int(window), float(window_bias),
+                           self.kb.data_ptr() if self.kb is not None else None,
+                           int(kb_block) if self.kb is not None else 0,
+                           int(self.kb.shape[1]) if self.kb is not None else 0)
+
+    @classmethod
+    def from_spec(cls, b, device="cuda"):
+        if b is None:
+            return None
+        return cls(b.sink_len, b.sink_bias, b.window, b.window_bias, b.kb_bias, b.kb_block, device)
+
+
+def _bias_ptr(bias: Optional[Bias]):
+    return ctypes.byref(bias.c) if bias is not None else None
+
+
+class Map:
+    """A compressed map: caller-owned device arrays described by an ``mr_bsr``."""
+
+    def __init__(self, H_s: int, L: int, block: int, dtype: int, capacity: int, device="cuda",
+                 store_mass: bool = False, store_lse: bool = False):
+        self.H_s, self.L, self.block, self.dtype, self.capacity = H_s, L, block, dtype, int(capacity)
+        self.nqb = L // block
+        self.nkw = (self.nqb + 31) // 32
+        n = H_s * self.nqb
+        dev = device
+        self.row_ptr = torch.zeros(n + 1, dtype=torch.int32, device=dev)
+        self.col_idx = torch.zeros(max(1, self.capacity), dtype=torch.int32, device=dev)
+        self.vals = torch.zeros((max(1, self.capacity), block, block), dtype=_torch_dtype(dtype), device=dev)
+        self.kept_mass = torch.zeros(n, dtype=torch.float32, device=dev)
+        self.kept_bits = torch.zeros((n, self.nkw), dtype=torch.int32, device=dev)
+        self.mass = torch.zeros((n, self.nqb), dtype=torch.float32, device=dev) if store_mass else None
+        self.lse = torch.zeros((H_s, L), dtype=torch.float32, device=dev) if store_lse else None
+        self.nnz = torch.zeros(1, dtype=torch.int64, device=dev)
+        self.c = BSR(H_s, L, block, dtype, self.capacity, self.row_ptr.data_ptr(), self.col_idx.data_ptr(),
+                     self.vals.data_ptr(), self.kept_mass.data_ptr(), self.kept_bits.data_ptr(),
+                     self.mass.data_ptr() if self.mass is not None else None,
+                     self.lse.data_ptr() if self.lse is not None else None, self.nnz.data_ptr())
+
+    def nnz_host(self, stream=None) -> int:
+        v = _c_i64(0)
+        check(LIB.mr_bsr_nnz(ctypes.byref(self.c), ctypes.byref(v), _stream(stream)), "mr_bsr_nnz")
+        return int(v.value)
+
+    def kept_bits_host(self) -> np.ndarray:
+        """Kept flags [H_s][nqb][nkb] as uint8 (host copy)."""
+        w = self.kept_bits.cpu().numpy().view(np.uint32).reshape(self.H_s, self.nqb, self.nkw)
+        bits = ((w[..., :, None] >> np.arange(32, dtype=np.uint32)) & 1).astype(np.uint8)
+        return bits.reshape(self.H_s, self.nqb, self.nkw * 32)[..., : self.nqb]
+
+    def export(self, n_tiles: Optional[int] = None, stream=None) -> torch.Tensor:
+        n = self.nnz_host(stream) if n_tiles is None else int(n_tiles)
+        n = min(n, self.capacity)
+        out = torch.empty((max(1, n), self.block, self.block), dtype=torch.float32, device=self.vals.device)
+        check(LIB.mr_bsr_export(ctypes.byref(self.c), n, out.data_ptr(), _stream(stream)), "mr_bsr_export")
+        return out[:n]
+
+
+def max_tiles(H_s: int, L: int, block: int) -> int:
+    return int(LIB.mr_bsr_max_tiles(H_s, L, block))
+
+
+def compress_workspace_bytes(H_s, L, d, block) -> int:
+    return int(LIB.mr_compress_workspace_bytes(H_s, L, d, block))
+
+
+def compress(Q: torch.Tensor, K: torch.Tensor, p: float, block: int, bias: Optional[Bias] = None,
+             scale: Optional[float] = None, capacity: Optional[int] = None, out: Optional[Map] = None,
+             ws: Optional[Workspace] = None, store_mass=False, store_lse=False, stream=None) -> Map:
+    """mr_compress: Q, K [H_s][L][d] (bf16 or fp32, CUDA) -> Map."""
+    _need_cuda(Q, K)
+    H, L, d = Q.shape
+    dt = _dt(Q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        cap = max_tiles(H, L, block) if capacity is None else capacity
+        out = Map(H, L, block, dt, cap, Q.device, store_mass, store_lse)
+    if ws is None:
+        ws = Workspace(compress_workspace_bytes(H, L, d, block), Q.device)
+    out.ws = ws
+    check(LIB.mr_compress(Q.data_ptr(), K.data_ptr(), dt, H, L, d, float(scale), float(p), _bias_ptr(bias),
+                          ctypes.byref(out.c), ws.ptr, ws.nbytes, _stream(stream)), "mr_compress")
+    return out
+
+
+def retrieve_workspace_bytes(m: Map, H_r: int, d_v: int, n_req: int) -> int:
+    return int(LIB.mr_retrieve_workspace_bytes(ctypes.byref(m.c), H_r, d_v, n_req))
+
+
+def retrieve(m: Map, W: torch.Tensor, V: torch.Tensor, out: Optional[torch.Tensor] = None,
+             v_req_off: Optional[torch.Tensor] = None, v_req_stride: Optional[int] = None,
+             v_head_stride: Optional[int] = None, n_req: Optional[int] = None,
+             ws: Optional[Workspace] = None, stream=None) -> torch.Tensor:
+    """mr_retrieve: W [H_r][H_s] fp32; V [H_r][L][d_v] or [n_req][H_r][L][d_v] (or a packed buffer
+    with explicit strides/offsets) -> O [n_req][H_r][L][d_v]."""
+    _need_cuda(W, V, v_req_off)
+    H_r = W.shape[0]
+    dt = _dt(V)
+    d_v = V.shape[-1]
+    if v_head_stride is None:
+        v_head_stride = V.shape[-2] * d_v
+    if n_req is None:
+        n_req = V.shape[0] if V.dim() == 4 else 1
+    if v_req_stride is None:
+        v_req_stride = H_r * v_head_stride
+    if out is None:
+        out = torch.empty((n_req, H_r, m.L, d_v), dtype=V.dtype, device=V.device)
+    _need_cuda(out)
+    if ws is None:
+        ws = Workspace(retrieve_workspace_bytes(m, H_r, d_v, n_req), V.device)
+    check(LIB.mr_retrieve(ctypes.byref(m.c), W.data_ptr(), H_r, V.data_ptr(), out.data_ptr(), dt, d_v, n_req,
+                          v_req_off.data_ptr() if v_req_off is not None else None, int(v_req_stride),
+                          int(v_head_stride), ws.ptr, ws.nbytes, _stream(stream)), "mr_retrieve")
+    return out
+
+
+def dense_ref(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, cu_q: torch.Tensor, cu_k: torch.Tensor,
+              q_offset: Optional[torch.Tensor], total_q: int, total_k: int, bias: Optional[Bias] = None,
+              scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+              ws: Optional[Workspace] = None, stream=None) -> torch.Tensor:
+    """mr_dense_ref: packed Q [H][total_q][d], K/V [H][total_k][d] -> O [H][total_q][d_v]."""
+    _need_cuda(Q, K, V, cu_q, cu_k, q_offset)
+    H, _, d = Q.shape
+    d_v = V.shape[-1]
+    n_seq = cu_q.shape[0] - 1
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((H, total_q, d_v), dtype=V.dtype, device=V.device)
+    if ws is None:
+        ws = Workspace(int(LIB.mr_dense_ref_workspace_bytes(n_seq)), Q.device)
+    check(LIB.mr_dense_ref(Q.data_ptr(), K.data_ptr(), V.data_ptr(), out.data_ptr(), _dt(Q), H, d, d_v,
+                           cu_q.data_ptr(), cu_k.data_ptr(),
+                           q_offset.data_ptr() if q_offset is not None else None, n_seq, int(total_q),
+                           int(total_k), float(scale), _bias_ptr(bias), ws.ptr, ws.nbytes, _stream(stream)),
+          "mr_dense_ref")
+    return out
+
+
+def profile_enable(on: bool = True) -> bool:
+    return bool(LIB.mr_profile_enable(1 if on else 0))
+
+
+def profile_read() -> dict:
+    """{kernel name: (total ms, launches)} for kernels launched since profiling was enabled."""
+    n = 64
+    ms = (ctypes.c_double * n)()
+    cnt = (_c_i64 * n)()
+    k = LIB.mr_profile_read(ctypes.cast(ms, _c_p), ctypes.cast(cnt, _c_p), n)
+    out = {}
+    for i in range(min(k, n)):
+        if cnt[i]:
+            out[LIB.mr_kernel_name(i).decode()] = (float(ms[i]), int(cnt[i]))
+    return out
+
+
+def kernel_launches() -> int:
+    return int(LIB.mr_kernel_launches())

@@ -1,0 +1,223 @@
+/*
+ * libmr: block-level top-p compression of causal attention maps and fused translated retrieval
+ * for cross-model attention-map reuse, on NVIDIA B200 (sm_100a).
+ *
+ * The method is MapFlow ("Accelerating Cross-Model LLM Inference via Attention Map Reuse"):
+ *   - a sender's per-head causal softmax maps are compressed once, per (layer, head, query
+ *     block), to the smallest set of key blocks whose probability mass reaches p, and stored in
+ *     Block Sparse Row form (sections 4 and 5.2, "Attention State Compressor");
+ *   - a receiver head's map is a non-negative, normalised linear mix of sender heads' maps
+ *     (section 3.3) and is applied to the receiver's values by one fused kernel that never writes
+ *     the translated map to global memory (section 5.4, "Attention Retrieval with Fused Kernel").
+ * mr_dense_ref is exact causal attention, softmax(QK^T/sqrt(d))V ("AttnCache Guide", section
+ * "The Quadratic Self-Attention Cost"), for rows that are not reused and as the p = 1 reference.
+ *
+ * Conventions for every entry point:
+ *   - All tensors are caller-owned device memory unless a parameter says "host".  The library
+ *     allocates no memory and frees nothing.
+ *   - Arguments are validated on the host before any launch; a rejected call returns
+ *     MR_ERR_INVALID_ARG or MR_ERR_UNSUPPORTED and launches nothing.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream) with no
+ *     host synchronisation.  Conditions found on the device (capacity overflow, a bounded wait
+ *     that ran out, a failed device check) are recorded in a status word inside the workspace;
+ *     read it with mr_sync_status.
+ *   - No exception crosses the ABI.  Device code never traps or asserts.
+ *   - Layouts are head-major and row-contiguous: element (h, row, c) of a [H][rows][dim]
+ *     tensor is at ((h * rows) + row) * dim + c.
+ */
+#ifndef MR_H_
+#define MR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MR_OK = 0,
+  MR_ERR_INVALID_ARG = 1,  /* null pointer, bad size or value (host check, nothing launched) */
+  MR_ERR_UNSUPPORTED = 2,  /* well-formed but outside this build: dtype, head dim, block, length */
+  MR_ERR_CAPACITY = 3,     /* the compressed map needs more tiles than capacity_tiles (device) */
+  MR_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  MR_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out; the kernel returned early */
+  MR_ERR_DEVICE_CHECK = 6, /* a device-side consistency check failed */
+  MR_ERR_RANGE = 7         /* a row's logits span too wide a range for the fp32 exponent path */
+} mr_status;
+
+typedef enum { MR_BF16 = 0, MR_F32 = 1 } mr_dtype;
+
+/*
+ * Synthetic causal logit bias b(h, i, j), added to sigma * q_i.k_j for j <= i.  It stands in for
+ * the attention-sink, local-window and retrieval-head patterns the AttnCache page describes
+ * ("The Attention Map Redundancy Discovery").  b is the MAXIMUM of the terms that apply, 0 when
+ * none applies:
+ *   sink_bias    when j < sink_len                (sink_len = 0 disables it)
+ *   window_bias  when i - j < window              (window = 0 disables it)
+ *   kb_bias[h * n_kb + j / kb_block]  when that device float is finite (-inf = no bias).
+ * For mr_dense_ref, i is the absolute position q_offset + row.  Pass NULL for "no bias".
+ */
+typedef struct {
+  int32_t sink_len;
+  float sink_bias;
+  int32_t window;
+  float window_bias;
+  const float* kb_bias; /* device [n_heads][n_kb] or NULL */
+  int32_t kb_block;     /* keys per kb_bias entry (> 0 when kb_bias != NULL) */
+  int32_t n_kb;         /* entries per head row (>= ceil(keys / kb_block)) */
+} mr_logit_bias;
+
+/*
+ * Block Sparse Row map of one layer's H_s sender heads (MapFlow section 4: "Block Sparse Row
+ * format").  Rows are (head h, query block I), numbered u = h * nqb + I with nqb = L / block;
+ * columns are key blocks J <= I, nkb = L / block, nkb_words = ceil(nkb / 32).
+ * The caller fills H_s, L, block, val_dtype, capacity_tiles and the pointers; mr_compress fills
+ * the arrays.
+ *   row_ptr   int32  [H_s * nqb + 1]  exclusive prefix sum of kept counts (row_ptr[0] = 0)
+ *   col_idx   int32  [capacity_tiles] kept key-block indices, ascending within each row
+ *   vals      [capacity_tiles][block][block] probabilities in val_dtype; tile t belongs to the
+ *             row u with row_ptr[u] <= t < row_ptr[u+1] and column col_idx[t]; element (a, b) of
+ *             a tile is the probability of query I*block + a on key J*block + b, stored
+ *             row-major (a * block + b); entries above the causal diagonal are 0.  Values are
+ *             not renormalised.
+ *   kept_mass float  [H_s * nqb]      mass of the kept blocks (fp64 sum, rounded to fp32)
+ *   kept_bits uint32 [H_s * nqb][nkb_words]  bit (J % 32) of word J / 32 set iff block J kept
+ *   mass      float  [H_s * nqb][nkb] optional block masses (NULL = not written); J > I is 0
+ *   lse       float  [H_s][L]         optional natural-log row normaliser log(sum_j exp(s_ij))
+ *   nnz       int64  [1]              number of kept tiles (may exceed capacity_tiles)
+ */
+typedef struct {
+  int32_t H_s;
+  int32_t L;
+  int32_t block;
+  mr_dtype val_dtype;
+  int64_t capacity_tiles;
+  int32_t* row_ptr;
+  int32_t* col_idx;
+  void* vals;
+  float* kept_mass;
+  uint32_t* kept_bits;
+  float* mass;
+  float* lse;
+  int64_t* nnz;
+} mr_bsr;
+
+/* Library version (major * 100 + minor). */
+int mr_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char* mr_status_string(mr_status s);
+
+/* 1 when the current device is sm_100 (B200-class) and the kernels can run, else 0. */
+int mr_device_supported(void);
+
+/*
+ * Workspace bytes mr_compress needs for this shape (device memory, 256-byte aligned, contents
+ * need no initialisation).  Returns 0 for an unsupported shape.
+ */
+size_t mr_compress_workspace_bytes(int H_s, int L, int d, int block);
+
+/*
+ * Worst-case tile count of a map of this shape: every causal tile kept,
+ * H_s * nqb * (nqb + 1) / 2.  A capacity of this size can never overflow.
+ */
+int64_t mr_bsr_max_tiles(int H_s, int L, int block);
+
+/*
+ * Compress one layer: MapFlow sections 4 and 5.2.
+ *   Q, K   [H_s][L][d] in dtype dt (MR_BF16: bf16; MR_F32: fp32)
+ *   scale  logit scale sigma (pass 1/sqrt(d) for standard attention)
+ *   p      top-p threshold in (0, 1]; p >= 1 keeps every causal block.  The kept set of row
+ *          (h, I) is the first k blocks of J = 0..I ordered by block mass descending (ties: the
+ *          smaller J first), k the least count whose cumulative mass (fp64) is >= p.
+ *          Block mass M_IJ = (1/block) * sum over the block's B x B probabilities.
+ *   bias   optional logit bias (NULL = none); kb_bias rows are per sender head.
+ *   out    map descriptor (see mr_bsr); out->H_s, L, block must equal the arguments.
+ *   ws     workspace of at least mr_compress_workspace_bytes(H_s, L, d, block) bytes.
+ * Supported: d in {64, 128}; block in {64, 128}; L a positive multiple of block with
+ * L / block <= 256; H_s <= 64.  MR_BF16 maps use bf16 vals; MR_F32 maps use fp32 vals.
+ * If the map needs more than capacity_tiles tiles, the status word records MR_ERR_CAPACITY and
+ * no tile at or beyond capacity_tiles is written (nnz still reports the full count).
+ */
+mr_status mr_compress(const void* Q, const void* K, mr_dtype dt, int H_s, int L, int d,
+                      float scale, float p, const mr_logit_bias* bias, mr_bsr* out, void* ws,
+                      size_t ws_bytes, void* stream);
+
+/* Workspace bytes mr_retrieve needs (device memory, 256-byte aligned). */
+size_t mr_retrieve_workspace_bytes(const mr_bsr* map, int H_r, int d_v, int n_req);
+
+/*
+ * Fused translated retrieval: MapFlow sections 3.3 and 5.4.
+ *   O_r[i] = sum_{j <= i} ( sum_s W[r][s] * A_s[i][j] * [key block of j kept for (s, block of i)] )
+ *            * V_r[j]
+ * for every receiver head r < H_r, query row i < map->L and request q < n_req.  The translated
+ * map is formed tile by tile on chip and never written to global memory.
+ *   map    a map filled by mr_compress (its vals dtype must equal dt)
+ *   W      device fp32 [H_r][H_s], row r = receiver head r's weights over sender heads
+ *   V      values in dtype dt: element (q, r, j, c) at
+ *          V + v_off(q) + r * v_head_stride + j * d_v + c,
+ *          v_off(q) = v_req_off[q] (device int64 array) or q * v_req_stride when v_req_off is NULL
+ *   O      output in dtype dt: element (q, r, i, c) at O + q * H_r * L * d_v + (r * L + i) * d_v + c
+ *   ws     workspace of at least mr_retrieve_workspace_bytes(map, H_r, d_v, n_req) bytes
+ * Supported: d_v in {64, 128}; H_r <= 256.
+ */
+mr_status mr_retrieve(const mr_bsr* map, const float* W, int H_r, const void* V, void* O,
+                      mr_dtype dt, int d_v, int n_req, const int64_t* v_req_off,
+                      int64_t v_req_stride, int64_t v_head_stride, void* ws, size_t ws_bytes,
+                      void* stream);
+
+/* Workspace bytes mr_dense_ref needs (device memory). */
+size_t mr_dense_ref_workspace_bytes(int n_seq);
+
+/*
+ * Exact causal attention over packed variable-length sequences ("AttnCache Guide": the
+ * standard softmax(QK^T * scale)V), with the same logit bias rule:
+ *   Q [H][total_q][d], K [H][total_k][d], V [H][total_k][d_v], O [H][total_q][d_v] (dtype dt)
+ *   cu_q, cu_k  device int32 [n_seq + 1] row offsets of each sequence in Q/O and K/V
+ *   q_offset    device int32 [n_seq] absolute position of each sequence's first query row
+ *               within its keys (NULL = 0): row i of sequence s attends keys
+ *               0 .. q_offset[s] + i, and requires q_offset[s] + len_q(s) <= len_k(s)
+ *   total_q, total_k  host ints equal to cu_q[n_seq] and cu_k[n_seq] (the per-head row
+ *               counts of the packed tensors; total_q also sizes the launch)
+ * Supported: d, d_v in {64, 128}.
+ */
+mr_status mr_dense_ref(const void* Q, const void* K, const void* V, void* O, mr_dtype dt, int H,
+                       int d, int d_v, const int32_t* cu_q, const int32_t* cu_k,
+                       const int32_t* q_offset, int n_seq, int total_q, int total_k, float scale,
+                       const mr_logit_bias* bias, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Synchronise `stream` and return the device-side status recorded in `ws` (MR_OK if nothing
+ * failed).  Every entry point that takes a workspace clears its status word when it is enqueued,
+ * so the result describes the most recent call that used `ws`.
+ */
+mr_status mr_sync_status(void* ws, void* stream);
+
+/* Synchronise `stream` and copy the map's kept-tile count to *nnz_host (host pointer). */
+mr_status mr_bsr_nnz(const mr_bsr* map, int64_t* nnz_host, void* stream);
+
+/*
+ * Convert the first n_tiles tiles of map->vals to fp32 row-major tiles
+ * ([n_tiles][block][block], element (a, b) = probability of query a on key b of the tile),
+ * whatever the internal storage order.  out is device memory.
+ */
+mr_status mr_bsr_export(const mr_bsr* map, int64_t n_tiles, float* out, void* stream);
+
+/*
+ * Measurement hooks (not part of the method).  When profiling is enabled, every entry point
+ * records a CUDA event on its stream before and after each kernel it launches; mr_profile_read
+ * waits for the recorded events and reports, per kernel id, the summed elapsed milliseconds and
+ * the launch count since profiling was enabled.  Kernel ids are stable small integers; their
+ * names come from mr_kernel_name (NULL past the last id).
+ */
+int mr_profile_enable(int on);      /* returns the previous state; enabling clears the records */
+int mr_profile_read(double* total_ms, int64_t* launches, int max_ids); /* host arrays; returns ids */
+const char* mr_kernel_name(int id);
+int64_t mr_kernel_launches(void);   /* kernels launched by this library in this process */
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MR_H_ */

@@ -1,0 +1,104 @@
+"""C-ABI checks that need no GPU: the library loads, exports what include/mr.h declares, sizes its
+workspaces, and rejects invalid calls on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mr.h")
+
+
+@pytest.fixture(scope="module")
+def mr():
+    from cross_model_attention_mr_b200 import mr as m
+    return m
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mr_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("mr_compress", "mr_retrieve", "mr_dense_ref", "mr_sync_status", "mr_bsr_export",
+                 "mr_status_string", "mr_compress_workspace_bytes", "mr_retrieve_workspace_bytes"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(mr):
+    lib = ctypes.CDLL(mr.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    # the binding declares a prototype for each of them
+    assert set(declared_functions()) <= set(mr.EXPORTS)
+
+
+def test_status_strings(mr):
+    for code in range(8):
+        s = mr.LIB.mr_status_string(code)
+        assert isinstance(s, bytes) and len(s) > 0
+    assert mr.LIB.mr_version() >= 100
+
+
+def test_workspace_sizes(mr):
+    assert mr.compress_workspace_bytes(32, 32768, 128, 128) > 32 * 32768 * 4
+    assert mr.compress_workspace_bytes(32, 32768, 96, 128) == 0       # unsupported head dim
+    assert mr.compress_workspace_bytes(32, 1000, 128, 64) == 0        # L not a multiple of the block
+    assert mr.compress_workspace_bytes(32, 64 * 257, 128, 64) == 0    # more than 256 key blocks
+    assert mr.max_tiles(32, 32768, 128) == 32 * 256 * 257 // 2
+    assert mr.max_tiles(4, 512, 64) == 4 * 8 * 9 // 2
+
+
+def _bsr(mr, H=4, L=512, B=64, dt=0, cap=100, fake=0x1000):
+    return mr.BSR(H, L, B, dt, cap, fake, fake, fake, fake, fake, None, None, fake)
+
+
+def test_compress_rejects_bad_arguments_without_launching(mr):
+    lib = mr.LIB
+    fake = 0x1000  # never dereferenced: every call below must fail validation first
+    ws_bytes = mr.compress_workspace_bytes(4, 512, 64, 64)
+    b = _bsr(mr)
+    call = lambda **kw: lib.mr_compress(kw.get("Q", fake), kw.get("K", fake), kw.get("dt", 0), kw.get("H", 4),
+                                        kw.get("L", 512), kw.get("d", 64), kw.get("scale", 0.125),
+                                        kw.get("p", 0.9), None, ctypes.byref(kw.get("b", b)), kw.get("ws", fake),
+                                        kw.get("wsb", ws_bytes), None)
+    assert call(Q=None) == mr.MR_ERR_INVALID_ARG
+    assert call(ws=None) == mr.MR_ERR_INVALID_ARG
+    assert call(dt=7) == mr.MR_ERR_INVALID_ARG
+    assert call(p=0.0) == mr.MR_ERR_INVALID_ARG
+    assert call(p=float("nan")) == mr.MR_ERR_INVALID_ARG
+    assert call(scale=float("inf")) == mr.MR_ERR_INVALID_ARG
+    assert call(d=96) == mr.MR_ERR_UNSUPPORTED
+    assert call(H=65, b=_bsr(mr, H=65)) == mr.MR_ERR_UNSUPPORTED
+    assert call(b=_bsr(mr, B=32)) == mr.MR_ERR_UNSUPPORTED
+    assert call(b=_bsr(mr, H=3)) == mr.MR_ERR_INVALID_ARG           # descriptor disagrees with H
+    assert call(b=_bsr(mr, dt=1)) == mr.MR_ERR_UNSUPPORTED          # vals dtype differs from inputs
+    assert call(b=_bsr(mr, cap=-1)) == mr.MR_ERR_INVALID_ARG
+    assert call(wsb=16) == mr.MR_ERR_INVALID_ARG
+    bad_bias = mr.LogitBias(0, 0.0, 0, 0.0, fake, 0, 8)             # kb table without a block size
+    assert lib.mr_compress(fake, fake, 0, 4, 512, 64, 0.125, 0.9, ctypes.byref(bad_bias), ctypes.byref(b),
+                           fake, ws_bytes, None) == mr.MR_ERR_INVALID_ARG
+
+
+def test_retrieve_and_dense_reject_bad_arguments(mr):
+    lib = mr.LIB
+    fake = 0x1000
+    b = _bsr(mr)
+    r = lambda **kw: lib.mr_retrieve(ctypes.byref(kw.get("b", b)), kw.get("W", fake), kw.get("H_r", 5), fake, fake,
+                                     kw.get("dt", 0), kw.get("dv", 64), kw.get("n", 1), None, 0,
+                                     kw.get("hs", 512 * 64), fake, 4096, None)
+    assert r(W=None) == mr.MR_ERR_INVALID_ARG
+    assert r(dv=80) == mr.MR_ERR_UNSUPPORTED
+    assert r(H_r=0) == mr.MR_ERR_INVALID_ARG
+    assert r(n=0) == mr.MR_ERR_INVALID_ARG
+    assert r(hs=10) == mr.MR_ERR_INVALID_ARG
+    assert r(dt=1) == mr.MR_ERR_UNSUPPORTED
+    d = lambda **kw: lib.mr_dense_ref(fake, fake, fake, fake, kw.get("dt", 0), 4, kw.get("d", 64), 64,
+                                      kw.get("cu", fake), fake, None, 2, 100, 100, 0.125, None, fake, 4096, None)
+    assert d(cu=None) == mr.MR_ERR_INVALID_ARG
+    assert d(d=32) == mr.MR_ERR_UNSUPPORTED
+    assert d(dt=3) == mr.MR_ERR_INVALID_ARG
