@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Benchmark of the attention-map-reuse hot path: prefill tokens/s for compress + retrieve at L=32K.
+
+One step = one pass of the whole path over one synthetic layer of the L=32768 workload
+(32 sender heads -> 64 receiver heads, d=128, bf16, block 128, p=0.9): block top-p compression of
+every sender head's causal map (mr_compress) followed by the fused translated retrieval for every
+receiver head (mr_retrieve).  value = tokens of all ranks / device time (max over ranks).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+For N > 1 it runs under torchrun, one rank per GPU; every rank compresses and retrieves its own
+independent sequence (weak scaling, no data-path collective).  ``--impl reference`` times the fp64
+CPU oracle on bounded samples of the same workload on the host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from cross_model_attention_mr_b200.workloads import config, draw_layers  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "prefill tokens/s for compress+retrieve at L=32K; % TC peak and % HBM peak"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", self.gpu], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_index_for(local_rank: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# ------------------------------------------------------------------------------------------------
+# algorithmic work of the path (what the method must do, independent of the implementation)
+# ------------------------------------------------------------------------------------------------
+def algorithmic(spec, nnz: int, union_tiles: int, n_req: int = 1):
+    B, d, L = spec.block, spec.d, spec.L
+    return {
+        # one causal QK^T per sender head: H_s * d * L * (L + 1) flops
+        "compress_flops": spec.H_s * d * L * (L + 1),
+        # the stored map: kept tiles of B*B bf16 probabilities plus one int32 column index each
+        "map_bytes": nnz * (B * B * 2 + 4),
+        # translated map times V over the union of kept key blocks, per receiver head and request
+        "retrieve_av_flops": spec.H_r * n_req * union_tiles * 2 * B * B * spec.d_v,
+        # head mixing: each kept sender tile is weighted into every receiver head
+        "retrieve_mix_flops": spec.H_r * nnz * 2 * B * B,
+    }
+
+
+def kernel_work(name: str, work: dict):
+    """(bound, amount, unit) of a kernel's algorithmic work per launch."""
+    if name in ("mr_compress_stats", "mr_compress_tc"):
+        return "tensor", work["compress_flops"], "flop"
+    if name in ("mr_emit", "mr_emit_tc"):
+        return "hbm", work["map_bytes"], "byte"
+    if name in ("mr_retrieve", "mr_retrieve_tc"):
+        return "tensor", work["retrieve_av_flops"] + work["retrieve_mix_flops"], "flop"
+    return None, 0, None
+
+
+def source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if its sources are unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        ent = d.get(kernel)
+        if not ent:
+            return None
+        if source_hash(ent["sources"]) != ent["source_hash"]:
+            return None
+        return float(ent["bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle timing (baseline / reference arm)
+# ------------------------------------------------------------------------------------------------
+def oracle_sample_time(spec, lay, units_I, rows, threads):
+    """Time the fp64 oracle on sampled compression units and retrieval rows and extrapolate to the
+    full step by exact per-unit work.  Returns (full-step seconds, description)."""
+    import oracle
+    B, L = spec.block, spec.L
+    nqb = L // B
+    units = [int((k * 7) % spec.H_s) * nqb + int(I) for k, I in enumerate(units_I)]
+    t0 = time.perf_counter()
+    r = oracle.compress(lay.Q, lay.K, spec.scale, float(np.float32(spec.p)), B, lay.bias, units=units,
+                        n_threads=threads)
+    tc = time.perf_counter() - t0
+    # work of a unit: B rows x (I+1)*B keys; total over all units of all heads
+    w_sample = sum((I + 1) for I in units_I)
+    w_total = spec.H_s * nqb * (nqb + 1) / 2
+    t_compress = tc * w_total / w_sample
+    kept = np.tril(np.ones((nqb, nqb), np.uint8))[None].repeat(spec.H_s, 0)
+    for u in units:
+        h, I = divmod(u, nqb)
+        kept[h, I] = r.kept[h, I]
+    t0 = time.perf_counter()
+    oracle.retrieve_rows(lay.Q, lay.K, spec.scale, B, kept, lay.W, lay.V, np.asarray(rows), lay.bias,
+                         n_threads=threads)
+    tr = time.perf_counter() - t0
+    t_retrieve = tr * (L * (L + 1) / 2) / sum(i + 1 for i in rows)
+    desc = (f"{len(units)} compression units (h, I) with I in {sorted(set(int(i) for i in units_I))} and "
+            f"{len(rows)} retrieval rows {list(map(int, rows))} of the L={L} workload, "
+            f"extrapolated by per-unit work ((I+1) key blocks per unit, (i+1) keys per row); "
+            f"sample took {tc + tr:.1f} s")
+    return t_compress + t_retrieve, desc, tc + tr
+
+
+def run_reference(args, spec, rank):
+    if rank != 0:
+        return
+    lay = draw_layers(spec)[0]
+    threads = os.cpu_count() or 1
+    nqb = spec.L // spec.block
+    rng = np.random.default_rng(11)
+    vals = []
+    desc = ""
+    for step in range(args.warmup + args.steps):
+        units_I = rng.integers(nqb // 2, nqb, size=threads).tolist()
+        rows = rng.integers(spec.L // 2, spec.L, size=max(1, threads // 4)).tolist()
+        t_full, desc, _ = oracle_sample_time(spec, lay, units_I, rows, threads)
+        if step >= args.warmup:
+            vals.append(spec.L / t_full)
+    value = float(statistics.median(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * spec.L / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": spec.name, "L": spec.L, "H_s": spec.H_s, "H_r": spec.H_r,
+                                        "d": spec.d, "block": spec.block, "p": spec.p},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": "per step: " + desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------------
+# native arm
+# ------------------------------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    spec = config(4)
+
+    if args.impl == "reference":
+        run_reference(args, spec, rank)
+        return
+
+    import torch
+    from cross_model_attention_mr_b200 import mr
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    if spec.seed is not None and rank:
+        from dataclasses import replace
+        spec = replace(spec, seed=spec.seed + 7919 * rank)  # independent sequence per rank
+
+    lay = draw_layers(spec)[0]
+    bf = torch.bfloat16
+    host = {
+        "Q": torch.from_numpy(lay.Q).to(bf).pin_memory(),
+        "K": torch.from_numpy(lay.K).to(bf).pin_memory(),
+        "V": torch.from_numpy(lay.V).to(bf).pin_memory(),
+        "W": torch.from_numpy(lay.W).pin_memory(),
+    }
+    Q, K, V, W = (host[k].cuda(non_blocking=True) for k in ("Q", "K", "V", "W"))
+    bias = mr.Bias.from_spec(lay.bias)
+    p = float(np.float32(spec.p))
+    cap = mr.max_tiles(spec.H_s, spec.L, spec.block)
+    m = mr.Map(spec.H_s, spec.L, spec.block, mr.MR_BF16, cap, "cuda")
+    ws_c = mr.Workspace(mr.compress_workspace_bytes(spec.H_s, spec.L, spec.d, spec.block))
+    ws_r = mr.Workspace(mr.retrieve_workspace_bytes(m, spec.H_r, spec.d_v, 1))
+    O = torch.empty((1, spec.H_r, spec.L, spec.d_v), dtype=bf, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        mr.compress(Q, K, p, spec.block, bias=bias, scale=spec.scale, out=m, ws=ws_c, stream=stream)
+        mr.retrieve(m, W, V, out=O, ws=ws_r, stream=stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st_c, st_r = ws_c.sync_status(), ws_r.sync_status()
+    if st_c or st_r:
+        raise SystemExit(f"device status compress={st_c} retrieve={st_r}")
+    nnz = m.nnz_host()
+    kept = m.kept_bits_host()
+    nqb = spec.L // spec.block
+    union_tiles = int(np.any(kept, axis=0).sum())
+    work = algorithmic(spec, nnz, union_tiles)
+
+    # ---- timed region (device time, CUDA events on the launching stream) ----
+    sampler = ClockSampler(gpu_index_for(local))
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    launches0 = mr.kernel_launches()
+    mr.profile_enable(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    prof = mr.profile_read()
+    mr.profile_enable(False)
+    launches = mr.kernel_launches() - launches0
+    ms = ev0.elapsed_time(ev1) / args.steps
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * spec.L / (ms / 1e3)
+
+    # ---- roofline of the dominant kernel ----
+    pk, pk_src = peaks()
+    dom = max(prof.items(), key=lambda kv: kv[1][0])
+    dname, (dms, dcnt) = dom
+    bound, amount, unit = kernel_work(dname, work)
+    avg_s = dms / dcnt / 1e3
+    if bound == "hbm":
+        achieved, peak, runit = amount / avg_s / 1e9, float(pk["hbm_gbs"]), "GB/s"
+    else:
+        achieved = amount / avg_s / 1e12
+        peak, runit = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])), "TFLOP/s"
+    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": runit, "frac": achieved / peak,
+                "traffic": traffic_for(dname), "kernel": dname, "peak_source": pk_src,
+                "peak_kind": "sustained" if bound != "hbm" else "copy"}
+    stages = {k: {"ms_per_launch": v[0] / v[1], "launches": v[1], "share": v[0] / sum(x[0] for x in prof.values())}
+              for k, v in prof.items()}
+
+    # ---- end to end through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        Oh = torch.empty(O.shape, dtype=bf).pin_memory()
+        h2d = sum(host[k].numel() * host[k].element_size() for k in host)
+        d2h = Oh.numel() * Oh.element_size()
+
+        def e2e_step():
+            for k, dst in (("Q", Q), ("K", K), ("V", V), ("W", W)):
+                dst.copy_(host[k], non_blocking=True)
+            step()
+            Oh.copy_(O, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        n_e2e = max(1, min(args.steps, 5))
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1) / n_e2e
+        if dist is not None:
+            t = torch.tensor([ems], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": world * spec.L / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": ems}
+
+    # ---- what the receiver would otherwise run: dense causal attention of its 64 heads ----
+    dense = None
+    if not args.no_dense:
+        import torch as _t
+        cu = _t.tensor([0, spec.L], dtype=_t.int32, device="cuda")
+        Qr = Q.repeat(2, 1, 1)[: spec.H_r].contiguous()  # receiver-shaped queries/keys (synthetic)
+        Kr = K.repeat(2, 1, 1)[: spec.H_r].contiguous()
+        Od = _t.empty_like(V)
+        ws_d = mr.Workspace(mr.LIB.mr_dense_ref_workspace_bytes(1))
+        mr.dense_ref(Qr, Kr, V, cu, cu, None, spec.L, spec.L, bias=None, scale=spec.scale, out=Od, ws=ws_d)
+        _t.cuda.synchronize()
+        d0, d1 = _t.cuda.Event(enable_timing=True), _t.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        mr.dense_ref(Qr, Kr, V, cu, cu, None, spec.L, spec.L, bias=None, scale=spec.scale, out=Od, ws=ws_d)
+        d1.record(stream)
+        _t.cuda.synchronize()
+        dms_ = d0.elapsed_time(d1)
+        dense = {"tokens_per_s": spec.L / (dms_ / 1e3), "ms": dms_, "heads": spec.H_r,
+                 "flops": 2 * spec.H_r * spec.L * (spec.L + 1) * (spec.d + spec.d_v) // 2}
+        del Qr, Kr, Od
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only) ----
+    cpu = None
+    if not args.no_cpu_baseline and world == 1 and rank == 0:
+        threads = os.cpu_count() or 1
+        # one large unit and one late row per core keeps the cores evenly loaded
+        units_I = [nqb - 1 - 3 * k for k in range(threads)]
+        rows = [spec.L - 1 - 977 * k for k in range(threads)]
+        t_full, desc, took = oracle_sample_time(spec, lay, units_I, rows, threads)
+        cpu = {"value": spec.L / t_full, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Gaussian Q/K/V, sink+window+retrieval-block logit bias, row-softmax W)",
+            "config": {"workload": spec.name, "L": spec.L, "H_s": spec.H_s, "H_r": spec.H_r, "d": spec.d,
+                       "d_v": spec.d_v, "block": spec.block, "p": spec.p, "layers": 1,
+                       "l2": "inputs larger than L2 (Q,K 268 MB each, V 537 MB, map %.1f GB)" % (work["map_bytes"] / 1e9),
+                       "parallelism": f"replicas{world}"},
+            "gpu_launches": int(launches),
+            "clocks": clocks,
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "stages": stages,
+            "map": {"nnz_tiles": nnz, "kept_fraction": nnz / (spec.H_s * nqb * (nqb + 1) / 2),
+                    "union_fraction": union_tiles / (nqb * (nqb + 1) / 2)},
+            "algorithmic": work,
+            "dense_ref": dense,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
