@@ -43,6 +43,8 @@ EXPORTS = {
     "mr_bsr_max_tiles": ([ctypes.c_int] * 3, _c_i64),
     "mr_compress": ([_c_p, _c_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _c_f32, _c_f32,
                      ctypes.POINTER(LogitBias), ctypes.POINTER(BSR), _c_p, _c_sz, _c_p], ctypes.c_int),
+    "mr_compress_noalloc": ([_c_p, _c_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _c_f32, _c_f32,
+                             ctypes.POINTER(LogitBias), ctypes.POINTER(BSR), _c_p], ctypes.c_int),
     "mr_retrieve_workspace_bytes": ([ctypes.POINTER(BSR), ctypes.c_int, ctypes.c_int, ctypes.c_int], _c_sz),
     "mr_retrieve": ([ctypes.POINTER(BSR), _c_p, ctypes.c_int, _c_p, _c_p, ctypes.c_int, ctypes.c_int,
                      ctypes.c_int, _c_p, _c_i64, _c_i64, _c_p, _c_sz, _c_p], ctypes.c_int),

@@ -144,6 +144,38 @@ mr_status mr_compress(const void* Q, const void* K, mr_dtype dt, int H_s, int L,
                       float scale, float p, const mr_logit_bias* bias, mr_bsr* out, void* ws,
                       size_t ws_bytes, void* stream);
 
+/*
+ * Allocation-free variant of mr_compress.  The paper has no counterpart: this is a deployment
+ * convenience of this library.
+ *
+ * Who needs it: callers that cannot allocate device memory, and so cannot hand mr_compress a
+ * workspace.  Examples are code running inside a framework whose memory pool already owns the
+ * GPU's memory (a raw allocation there fails or fragments the pool), plug-ins held to a fixed,
+ * pre-planned memory budget, and serving loops that must not call the allocator once running.
+ *
+ * It computes exactly what mr_compress computes, with the same arguments except the workspace.
+ * The scratch comes from one fixed array compiled into the library, of
+ * MR_COMPRESS_NOALLOC_SCRATCH_BYTES bytes.  Every GPU that loads the library holds that array
+ * until the process exits.  The call allocates and frees nothing; the caller still owns Q, K and
+ * every array of *out.
+ *   - Limit: shapes with mr_compress_workspace_bytes(H_s, L, d, out->block) larger than the array
+ *     are rejected with MR_ERR_UNSUPPORTED before any work is enqueued.  That allows
+ *     H_s * L <= 1048576 rows and H_s * (L / block) <= 16384 query blocks, e.g. 32 heads of 32768
+ *     tokens.
+ *   - First call on a device: it looks up the array's device address with that device current.
+ *     Make the first call on each device before any stream capture begins.
+ *   - All calls share the one array, which keeps the last call's contents.  Each call clears the
+ *     parts that must start at zero, in stream order.  Calls whose work can overlap on the GPU
+ *     (other streams or other host threads without ordering between them) race on the array and
+ *     corrupt each other's maps: order them.
+ *   - There is no caller-visible workspace, so mr_sync_status cannot read this call's status
+ *     word.  A map that outgrew its capacity shows as *out->nnz > out->capacity_tiles.
+ */
+#define MR_COMPRESS_NOALLOC_SCRATCH_BYTES (256 + 4194304 + 65536)
+mr_status mr_compress_noalloc(const void* Q, const void* K, mr_dtype dt, int H_s, int L, int d,
+                              float scale, float p, const mr_logit_bias* bias, mr_bsr* out,
+                              void* stream);
+
 /* Workspace bytes mr_retrieve needs (device memory, 256-byte aligned). */
 size_t mr_retrieve_workspace_bytes(const mr_bsr* map, int H_r, int d_v, int n_req);
 
