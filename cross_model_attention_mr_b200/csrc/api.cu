@@ -171,7 +171,7 @@ mr_status mr_retrieve(const mr_bsr* map, const float* W, int H_r, const void* V,
   a.v_head_stride = v_head_stride;
   a.ws = (WsHeader*)ws;
   a.stream = st;
-  return from_cuda(simt_retrieve(a));
+  return from_cuda(tc_retrieve_supported(a) ? tc_retrieve(a) : simt_retrieve(a));
 }
 
 size_t mr_dense_ref_workspace_bytes(int n_seq) {

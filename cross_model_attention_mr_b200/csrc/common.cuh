@@ -70,6 +70,28 @@ __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
+// Storage order of a B x B map tile (see mr_bsr.vals): the tile is split into panels of
+// 128 bytes of columns (P = 128 / sizeof(T) columns); each panel stores its B rows one after the
+// other, 128 bytes per row, and inside a row the 16-byte chunk c sits at chunk position
+// c ^ (row % 8).  A panel is therefore exactly a 128-byte-swizzled K-major MMA operand and can be
+// read by 8 consecutive rows without shared-memory bank conflicts.
+template <typename T>
+__host__ __device__ __forceinline__ int tile_offset(int a, int b, int B) {
+  constexpr int P = 128 / (int)sizeof(T), E = 16 / (int)sizeof(T);
+  const int panel = b / P, c = (b % P) / E;
+  return panel * B * P + a * P + ((c ^ (a & 7)) * E) + (b % E);
+}
+
+// Inverse of tile_offset: row a and column b of the element stored at offset p.
+template <typename T>
+__host__ __device__ __forceinline__ void tile_coords(int p, int B, int& a, int& b) {
+  constexpr int P = 128 / (int)sizeof(T), E = 16 / (int)sizeof(T);
+  const int panel = p / (B * P), rem = p - panel * B * P;
+  a = rem / P;
+  const int pc = (rem % P) / E;
+  b = panel * P + ((pc ^ (a & 7)) * E) + (rem % E);
+}
+
 // Rank of key block J among the kept blocks of one row: number of kept blocks below J.
 __device__ __forceinline__ int kept_rank(const uint32_t* bits, int J) {
   int r = 0;

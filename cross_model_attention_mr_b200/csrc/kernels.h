@@ -58,6 +58,10 @@ cudaError_t simt_compress(const CompressArgs& a);
 cudaError_t simt_retrieve(const RetrieveArgs& a);
 cudaError_t simt_dense(const DenseArgs& a);
 
+// Tensor-core kernels (bf16, sm_100a).
+bool tc_retrieve_supported(const RetrieveArgs& a);
+cudaError_t tc_retrieve(const RetrieveArgs& a);
+
 // Shared by every compress path: exclusive scan of the kept counts into row_ptr, nnz, capacity.
 cudaError_t launch_scan_counts(const int* count, int n, mr_bsr map, WsHeader* ws, cudaStream_t st);
 

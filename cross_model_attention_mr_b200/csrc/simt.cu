@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(kThreads) k_emit(
           const int c = tx + 16 * b;
           const int j = J * BLK + c;
           const float pr = (j <= i) ? expf(S[a][b] * scale + bias_term(bias, h, i, j) - lse_s[r]) : 0.f;
-          out[r * BLK + c] = from_f32<TV>(pr);
+          out[tile_offset<TV>(r, c, BLK)] = from_f32<TV>(pr);
         }
       }
       if (tid == 0) col_idx[t] = J;
@@ -299,8 +299,9 @@ __global__ void __launch_bounds__(kThreads) k_retrieve(
     __syncthreads();
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      const int idx = tid + e * kThreads;
-      Xs[(idx / BLK) * (BLK + 1) + (idx % BLK)] = x[e];
+      int ra, cb;
+      tile_coords<T>(tid + e * kThreads, BLK, ra, cb);
+      Xs[ra * (BLK + 1) + cb] = x[e];
     }
     load_rows<T, BLK, DV>(Vs, Vr + (size_t)J * BLK * DV, BLK);
     __syncthreads();
@@ -476,9 +477,13 @@ __global__ void k_scan_counts(const int* __restrict__ count, int n, int32_t* __r
 }
 
 template <typename TV>
-__global__ void k_export(const TV* __restrict__ vals, int64_t n_elems, float* __restrict__ out) {
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n_elems; e += (int64_t)gridDim.x * blockDim.x)
-    out[e] = to_f32(vals[e]);
+__global__ void k_export(const TV* __restrict__ vals, int64_t n_elems, int B, float* __restrict__ out) {
+  const int64_t tsz = (int64_t)B * B;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n_elems; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = e / tsz;
+    const int w = (int)(e - t * tsz);
+    out[e] = to_f32(vals[t * tsz + tile_offset<TV>(w / B, w % B, B)]);
+  }
 }
 
 template <typename KernelT>
@@ -585,9 +590,9 @@ cudaError_t launch_export(const mr_bsr& map, int64_t n_tiles, float* out, cudaSt
   const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
   ProfScope ps(kKExport, st);
   if (map.val_dtype == MR_BF16)
-    k_export<__nv_bfloat16><<<blocks, 256, 0, st>>>((const __nv_bfloat16*)map.vals, n, out);
+    k_export<__nv_bfloat16><<<blocks, 256, 0, st>>>((const __nv_bfloat16*)map.vals, n, map.block, out);
   else
-    k_export<float><<<blocks, 256, 0, st>>>((const float*)map.vals, n, out);
+    k_export<float><<<blocks, 256, 0, st>>>((const float*)map.vals, n, map.block, out);
   return cudaGetLastError();
 }
 

@@ -76,11 +76,16 @@ typedef struct {
  * the arrays.
  *   row_ptr   int32  [H_s * nqb + 1]  exclusive prefix sum of kept counts (row_ptr[0] = 0)
  *   col_idx   int32  [capacity_tiles] kept key-block indices, ascending within each row
- *   vals      [capacity_tiles][block][block] probabilities in val_dtype; tile t belongs to the
- *             row u with row_ptr[u] <= t < row_ptr[u+1] and column col_idx[t]; element (a, b) of
- *             a tile is the probability of query I*block + a on key J*block + b, stored
- *             row-major (a * block + b); entries above the causal diagonal are 0.  Values are
- *             not renormalised.
+ *   vals      [capacity_tiles][block * block] probabilities in val_dtype; tile t belongs to
+ *             the row u with row_ptr[u] <= t < row_ptr[u+1] and column col_idx[t]; element (a, b)
+ *             of a tile is the probability of query I*block + a on key J*block + b; entries above
+ *             the causal diagonal are 0.  Values are not renormalised.  Storage order inside a
+ *             tile: panels of P = 128 / sizeof(element) columns, each panel holding its `block`
+ *             rows of 128 bytes in turn; in row a, the 16-byte chunk c of the panel is stored at
+ *             chunk position c ^ (a % 8).  So element (a, b) sits at
+ *               (b / P) * block * P + a * P + E * (((b % P) / E) ^ (a % 8)) + b % E,
+ *             E = 16 / sizeof(element).  (Each panel is a 128-byte-swizzled MMA operand.)
+ *             mr_bsr_export converts tiles to plain row-major fp32.
  *   kept_mass float  [H_s * nqb]      mass of the kept blocks (fp64 sum, rounded to fp32)
  *   kept_bits uint32 [H_s * nqb][nkb_words]  bit (J % 32) of word J / 32 set iff block J kept
  *   mass      float  [H_s * nqb][nkb] optional block masses (NULL = not written); J > I is 0
