@@ -130,7 +130,10 @@ mr_status mr_compress(const void* Q, const void* K, mr_dtype dt, int H_s, int L,
   a.count_ws = (int*)((char*)ws + lay.count_off);
   a.map = *out;
   a.stream = st;
-  return from_cuda(simt_compress(a));
+  if (!tc_compress_supported(a)) return from_cuda(simt_compress(a));
+  if ((e = tc_compress_stats(a)) != cudaSuccess) return MR_ERR_CUDA;
+  if ((e = launch_scan_counts(a.count_ws, H_s * (L / out->block), a.map, a.ws, st)) != cudaSuccess) return MR_ERR_CUDA;
+  return from_cuda(tc_emit(a));
 }
 
 size_t mr_retrieve_workspace_bytes(const mr_bsr* map, int H_r, int d_v, int n_req) {

@@ -1,0 +1,364 @@
+// Emit the kept tiles of the compressed map on sm_100a (bf16 Q/K, d = 128): MapFlow section 5.2,
+// "stores retained attention blocks in BSR format".
+//
+// After the statistics pass and the scan of kept counts, every kept tile (h, I, J) is recomputed:
+// S = Q_I K_J^T on the tensor core, P_ij = 2^(s'_ij - lse2_i) (s' the biased logit in base 2,
+// lse2 the row log-normaliser; zero above the causal diagonal), rounded to bf16 and written in
+// the map's storage order (128-byte swizzled panels) to its BSR position.  Tiles that no query
+// block of the unit kept are neither loaded nor multiplied.  Each tile leaves shared memory with
+// one bulk store, so the pass is bound by the HBM write of the map.
+//
+// Roles per CTA (persistent, units longest-first): TMA producer warp (Q rows, ring of needed K
+// tiles), MMA warp (128 x 128 tiles into two Tensor Memory buffers), two warpgroups that take
+// alternate needed tiles (one query row per thread).  All waits are bounded.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "profile.h"
+#include "sm100.cuh"
+#include "tma_host.h"
+
+namespace mr {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 384;
+constexpr int kProducerWarp = 0;
+constexpr int kMmaWarp = 1;
+constexpr int kSoftmaxWarp0 = 4;
+constexpr int kKStages = 3;
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct Params {
+  int H, L, B, nqb, nkw, n_rb, n_units;
+  float a;
+  Bias bias;
+  const float* lse_ws;
+  const int32_t* row_ptr;
+  const uint32_t* kept_bits;
+  int64_t capacity;
+  int32_t* col_idx;
+  __nv_bfloat16* vals;
+  WsHeader* ws;
+};
+
+struct Smem {
+  __nv_bfloat16 q[2][128 * 64];
+  __nv_bfloat16 k[kKStages][2][128 * 64];
+  __nv_bfloat16 stage[2][128 * 128];  // per warpgroup: one tile in storage order
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+  int wg_fail[2];  // written by a warpgroup's warps only before a barrier, read after it
+};
+
+__device__ __forceinline__ void fail(Smem& s, const Params& p, uint32_t detail) {
+  set_status(p.ws, MR_ERR_TIMEOUT, detail);
+  s.abort = 1;
+}
+
+__device__ __forceinline__ void unit_of(const Params& p, int k, int& h, int& rb) {
+  rb = p.n_rb - 1 - k / p.H;
+  h = k % p.H;
+}
+
+__device__ __forceinline__ bool kept(const Params& p, int h, int I, int J) {
+  if (I < 0 || I >= p.nqb || J > I) return false;
+  return (__ldg(p.kept_bits + (size_t)(h * p.nqb + I) * p.nkw + (J >> 5)) >> (J & 31)) & 1u;
+}
+
+// Which 64 x 64 (B = 64) or 128 x 128 (B = 128) pieces of key tile T the unit emits:
+// bit (2 * rowhalf + colhalf) for B = 64, bit 0 for B = 128.
+__device__ __forceinline__ uint32_t tile_pieces(const Params& p, int h, int rb, int T) {
+  if (p.B == 128) return kept(p, h, rb, T) ? 1u : 0u;
+  uint32_t m = 0;
+  for (int rh = 0; rh < 2; ++rh)
+    for (int ch = 0; ch < 2; ++ch)
+      if (kept(p, h, 2 * rb + rh, 2 * T + ch)) m |= 1u << (2 * rh + ch);
+  return m;
+}
+
+__device__ void producer(Smem& s, const Params& p, const CUtensorMap* tq, const CUtensorMap* tk) {
+  if ((threadIdx.x & 31) != 0) return;
+  uint32_t nk = 0, nu = 0;
+  bool ok = true;
+  for (int k = blockIdx.x; k < p.n_units && ok; k += gridDim.x, ++nu) {
+    int h, rb;
+    unit_of(p, k, h, rb);
+    if (nu > 0 && !mbar_wait(&s.q_empty, (nu - 1) & 1, &s.abort, kTimeoutNs)) {
+      fail(s, p, 0x501);
+      break;
+    }
+    const int qrow = h * p.L + 128 * rb;
+    mbar_arrive_expect_tx(&s.q_full, 2 * 128 * 64 * 2);
+    tma_load_2d(&s.q[0][0], tq, &s.q_full, 0, qrow);
+    tma_load_2d(&s.q[1][0], tq, &s.q_full, 64, qrow);
+    for (int T = 0; T <= rb; ++T) {
+      if (!tile_pieces(p, h, rb, T)) continue;
+      const int st = (int)(nk % kKStages);
+      if (nk >= (uint32_t)kKStages && !mbar_wait(&s.k_empty[st], ((nk / kKStages) - 1) & 1, &s.abort, kTimeoutNs)) {
+        fail(s, p, 0x502);
+        ok = false;
+        break;
+      }
+      const int krow = h * p.L + 128 * T;
+      mbar_arrive_expect_tx(&s.k_full[st], 2 * 128 * 64 * 2);
+      tma_load_2d(&s.k[st][0][0], tk, &s.k_full[st], 0, krow);
+      tma_load_2d(&s.k[st][1][0], tk, &s.k_full[st], 64, krow);
+      ++nk;
+    }
+  }
+  const int never = 0;
+  for (uint32_t g = (nk > (uint32_t)kKStages ? nk - kKStages : 0); g < nk; ++g)
+    mbar_wait(&s.k_full[g % kKStages], (g / kKStages) & 1, &never, kTimeoutNs);
+  if (nu > 0) mbar_wait(&s.q_full, (nu - 1) & 1, &never, kTimeoutNs);
+}
+
+__device__ void mma_issuer(Smem& s, const Params& p) {
+  if ((threadIdx.x & 31) != 0) return;
+  const uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+  const uint32_t tbase = s.tmem_base;
+  uint32_t nk = 0, nu = 0, nb[2] = {0, 0};
+  bool ok = true;
+  for (int k = blockIdx.x; k < p.n_units && ok; k += gridDim.x, ++nu) {
+    int h, rb;
+    unit_of(p, k, h, rb);
+    if (!mbar_wait(&s.q_full, nu & 1, &s.abort, kTimeoutNs)) {
+      fail(s, p, 0x511);
+      break;
+    }
+    int n_local = 0;
+    for (int T = 0; T <= rb; ++T) {
+      if (!tile_pieces(p, h, rb, T)) continue;
+      const int st = (int)(nk % kKStages), b = n_local & 1;
+      if (!mbar_wait(&s.k_full[st], (nk / kKStages) & 1, &s.abort, kTimeoutNs) ||
+          (nb[b] > 0 && !mbar_wait(&s.s_empty[b], (nb[b] - 1) & 1, &s.abort, kTimeoutNs))) {
+        fail(s, p, 0x512);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t qa[2] = {smem_u32(&s.q[0][0]), smem_u32(&s.q[1][0])};
+      const uint32_t ka[2] = {smem_u32(&s.k[st][0][0]), smem_u32(&s.k[st][1][0])};
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t da = sdesc_sw128(qa[kk >> 2] + 32 * (kk & 3), 16, 1024);
+        const uint64_t db = sdesc_sw128(ka[kk >> 2] + 32 * (kk & 3), 16, 1024);
+        mma_bf16_ss(tbase + 128 * b, da, db, idesc, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(&s.s_full[b]);
+      mma_commit(&s.k_empty[st]);
+      ++nb[b];
+      ++nk;
+      ++n_local;
+    }
+    if (ok) mma_commit(&s.q_empty);
+  }
+  mma_commit(&s.mma_done);
+  const int never = 0;
+  mbar_wait(&s.mma_done, 0, &never, kTimeoutNs);
+}
+
+__device__ __forceinline__ float kb_offset(const Bias& b, int h, int j) {
+  if (b.kb == nullptr) return 0.f;
+  const float v = __ldg(b.kb + (size_t)h * b.n_kb + j / b.kb_block);
+  return v == -INFINITY ? 0.f : v * kLog2e;
+}
+
+__device__ void emit_group(Smem& s, const Params& p, int w) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q4 = warp & 3;
+  const int row = 32 * q4 + lane;
+  const int gtid = threadIdx.x - 32 * (kSoftmaxWarp0 + 4 * w);
+  const uint32_t tbase = s.tmem_base;
+  const uint32_t lane_addr = (uint32_t)(32 * q4) << 16;
+  const uint32_t bar_id = 2 + w;
+  char* stage = reinterpret_cast<char*>(&s.stage[w][0]);
+  uint32_t nb = 0;
+  bool ok = true;
+  bool store_pending = false;
+  for (int k = blockIdx.x; k < p.n_units && ok; k += gridDim.x) {
+    int h, rb;
+    unit_of(p, k, h, rb);
+    const int i = 128 * rb + row;
+    const bool row_ok = i < p.L;
+    const float lse2 = row_ok ? __ldg(p.lse_ws + (size_t)h * p.L + i) * kLog2e : 0.f;
+    const int rh = row >> 6;  // B = 64: which query block of the unit this row belongs to
+    int n_local = 0;
+    for (int T = 0; T <= rb && ok; ++T) {
+      const uint32_t pieces = tile_pieces(p, h, rb, T);
+      if (!pieces) continue;
+      const int mine = n_local++ & 1;
+      if (mine != w) continue;
+      if (!mbar_wait(&s.s_full[w], nb & 1, &s.abort, kTimeoutNs)) {
+        fail(s, p, 0x521);
+        s.wg_fail[w] = 1;
+      }
+      ++nb;
+      tc_fence_after();
+      // the staging buffer may still be read by this warpgroup's previous bulk store
+      if (gtid == 0 && store_pending) bulk_wait_read<0>();
+      named_sync(bar_id, 128);
+      // every warp of the warpgroup takes the same decision and passes the same barriers
+      const bool stop = s.wg_fail[w] != 0;
+      const int j_tile = 128 * T;
+      const bool special = (T == rb) || (j_tile < p.bias.sink_len) ||
+                           (p.bias.window > 0 && j_tile + 127 > 128 * rb - p.bias.window);
+      // which 64-key halves of this row's tile are stored
+      const uint32_t row_mask = p.B == 128 ? 3u : ((pieces >> (2 * rh)) & 3u);
+#pragma unroll
+      for (int hh = 0; hh < 2 && !stop; ++hh) {
+        uint32_t raw[2][32];
+        tmem_ld32(tbase + lane_addr + 128 * w + 64 * hh, raw[0]);
+        tmem_ld32(tbase + lane_addr + 128 * w + 64 * hh + 32, raw[1]);
+        tmem_wait_ld();
+        if (hh == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.s_empty[w]);
+        }
+        if (!((row_mask >> hh) & 1u)) continue;  // warp-uniform
+        // destination: panel hh (B = 128) or the 64 x 64 piece (rh, hh) (B = 64)
+        char* dst = p.B == 128 ? stage + 16384 * hh + row * 128 : stage + 8192 * (2 * rh + hh) + (row & 63) * 128;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int j0 = j_tile + 64 * hh + 32 * cc;
+          float pr[32];
+          if (!special) {
+            const float o = kb_offset(p.bias, h, j0) - lse2;
+#pragma unroll
+            for (int t = 0; t < 32; ++t) pr[t] = ex2_approx(fmaf(__uint_as_float(raw[cc][t]), p.a, o));
+          } else {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+              const int j = j0 + t;
+              pr[t] = (row_ok && j <= i)
+                          ? ex2_approx(fmaf(__uint_as_float(raw[cc][t]), p.a, bias_term(p.bias, h, i, j) * kLog2e) - lse2)
+                          : 0.f;
+            }
+          }
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(pr[8 * c8 + 2 * e], pr[8 * c8 + 2 * e + 1]);
+              pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            const int chunk = 4 * cc + c8;  // 16-byte chunk within the 64-column panel row
+            *reinterpret_cast<uint4*>(dst + ((chunk ^ (row & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      named_sync(bar_id, 128);
+      if (stop) {
+        ok = false;
+        break;
+      }
+      if (gtid == 0) {
+        // one bulk store per stored tile (B = 128) or 64 x 64 piece (B = 64)
+        for (int piece = 0; piece < (p.B == 128 ? 1 : 4); ++piece) {
+          if (!((pieces >> piece) & 1u)) continue;
+          const int I = p.B == 128 ? rb : 2 * rb + (piece >> 1);
+          const int J = p.B == 128 ? T : 2 * T + (piece & 1);
+          const int u = h * p.nqb + I;
+          const int64_t t = (int64_t)__ldg(p.row_ptr + u) + kept_rank(p.kept_bits + (size_t)u * p.nkw, J);
+          if (t >= p.capacity) continue;
+          const int64_t tbytes = (int64_t)p.B * p.B * 2;
+          bulk_s2g(reinterpret_cast<char*>(p.vals) + t * tbytes, stage + (p.B == 128 ? 0 : 8192 * piece),
+                   (uint32_t)tbytes);
+          p.col_idx[t] = J;
+        }
+        bulk_commit();
+        store_pending = true;
+      }
+    }
+  }
+  if (gtid == 0 && store_pending) bulk_wait_all<0>();
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_emit_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk, Params p) {
+  extern __shared__ unsigned char smem_raw[];
+  Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(&s.q_full, 1);
+    mbar_init(&s.q_empty, 1);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(&s.k_full[i], 1);
+      mbar_init(&s.k_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.s_full[i], 1);
+      mbar_init(&s.s_empty[i], 4);
+    }
+    mbar_init(&s.mma_done, 1);
+    s.abort = 0;
+    s.wg_fail[0] = s.wg_fail[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&s.tmem_base, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kProducerWarp)
+    producer(s, p, &tq, &tk);
+  else if (warp == kMmaWarp)
+    mma_issuer(s, p);
+  else if (warp >= kSoftmaxWarp0)
+    emit_group(s, p, (warp - kSoftmaxWarp0) >> 2);
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(s.tmem_base, 256);
+}
+
+}  // namespace
+
+cudaError_t tc_emit(const CompressArgs& a) {
+  Params p;
+  p.H = a.H;
+  p.L = a.L;
+  p.B = a.block;
+  p.nqb = a.L / a.block;
+  p.nkw = (p.nqb + 31) / 32;
+  p.n_rb = (a.L + 127) / 128;
+  p.n_units = p.H * p.n_rb;
+  p.a = a.scale * kLog2e;
+  p.bias = a.bias;
+  p.lse_ws = a.lse_ws;
+  p.row_ptr = a.map.row_ptr;
+  p.kept_bits = a.map.kept_bits;
+  p.capacity = a.map.capacity_tiles;
+  p.col_idx = a.map.col_idx;
+  p.vals = (__nv_bfloat16*)a.map.vals;
+  p.ws = a.ws;
+  CUtensorMap tq, tk;
+  const uint64_t rows = (uint64_t)a.H * a.L;
+  if (!make_tmap_bf16_2d(&tq, a.Q, 128, rows, 256, 64, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tk, a.K, 128, rows, 256, 64, 128)) return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = p.n_units < sms ? p.n_units : sms;
+  const size_t smem = sizeof(Smem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(k_emit_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  ProfScope ps(kKEmitTc, a.stream);
+  k_emit_tc<<<grid, kThreads, smem, a.stream>>>(tq, tk, p);
+  return cudaGetLastError();
+}
+
+}  // namespace mr

@@ -55,10 +55,14 @@ struct DenseArgs {
 
 // SIMT (CUDA-core) kernels: fp32 inputs, and bf16 where no tensor-core kernel applies.
 cudaError_t simt_compress(const CompressArgs& a);
+cudaError_t simt_emit(const CompressArgs& a);  // emit pass only (after statistics and scan)
 cudaError_t simt_retrieve(const RetrieveArgs& a);
 cudaError_t simt_dense(const DenseArgs& a);
 
 // Tensor-core kernels (bf16, sm_100a).
+bool tc_compress_supported(const CompressArgs& a);
+cudaError_t tc_compress_stats(const CompressArgs& a);  // row normalisers, masses, selection
+cudaError_t tc_emit(const CompressArgs& a);            // kept tiles -> map storage
 bool tc_retrieve_supported(const RetrieveArgs& a);
 cudaError_t tc_retrieve(const RetrieveArgs& a);
 

@@ -53,10 +53,18 @@ struct Params {
   WsHeader* ws;
 };
 
+// What a ring slot holds, written by the producer before the slot's full barrier is armed.
+struct SlotMeta {
+  float w[kAcc];   // W[r][s] of the unit's receiver heads for the slot's sender head s
+  uint32_t flags;  // kHalf0 | kHalf1 | kLastSub | kLastUnit | kEmptyUnit
+};
+constexpr uint32_t kHalf0 = 1u, kHalf1 = 2u, kLastSub = 4u, kLastUnit = 8u, kEmptyUnit = 16u;
+
 struct Smem {
   __nv_bfloat16 slot[kSlots][kSlotBytes / 2];
   __nv_bfloat16 x[kAcc][128 * 64];
   __nv_bfloat16 v[kAcc][64 * 128];
+  SlotMeta meta[kSlots];
   uint64_t slot_full[kSlots];
   uint64_t slot_empty[kSlots];
   uint64_t x_full, x_empty, v_full, v_empty, o_full, o_empty, mma_done;
@@ -112,15 +120,44 @@ __device__ __forceinline__ void fail(Smem& s, const Params& p, uint32_t detail) 
 }
 
 // ------------------------------------------------------------------------------------------------
+// Per-lane view of one (sender head, query block) map row while J advances within a unit: the
+// current 32-bit word of kept bits, the number of kept blocks below J, and the row's first tile.
+struct RowCursor {
+  const uint32_t* bits;
+  uint32_t word;
+  int count;
+  int64_t first;
+  bool live;
+  __device__ __forceinline__ void start(const Params& p, int s, int I) {
+    live = s < p.H_s && I >= 0;
+    count = 0;
+    if (live) {
+      const int row = s * p.nqb + I;
+      bits = p.kept_bits + (size_t)row * p.nkw;
+      word = __ldg(bits);
+      first = __ldg(p.row_ptr + row);
+    } else {
+      bits = nullptr;
+      word = 0u;
+      first = 0;
+    }
+  }
+  // kept flag of block J (J visited in increasing order, J <= I of the row)
+  __device__ __forceinline__ bool at(int J) {
+    if (!live) return false;
+    if ((J & 31) == 0 && J > 0) word = __ldg(bits + (J >> 5));
+    return (word >> (J & 31)) & 1u;
+  }
+};
+
 template <int G>
 __device__ void producer(Smem& s, const Params& p, const CUtensorMap* tmap_v) {
   const int lane = threadIdx.x & 31;
-  uint32_t f = 0;        // slot fills issued
-  uint32_t nv = 0;       // V fills issued (one per executed sub-step)
+  uint32_t f = 0;   // slot fills issued
+  uint32_t nv = 0;  // V fills issued (one per executed sub-step)
   const int nparts = p.B / 64;
   bool ok = true;
 
-  // Load V rows j0..j0+63 of every (head, request) accumulator of unit u for sub-step `n`.
   auto issue_v = [&](const Unit& u, int j0) {
     uint32_t bytes = 0;
     for (int a = 0; a < G * p.R; ++a)
@@ -137,84 +174,152 @@ __device__ void producer(Smem& s, const Params& p, const CUtensorMap* tmap_v) {
     ++nv;
   };
 
+  // claim the next ring slot (lane 0 waits), returns false on timeout
+  auto claim = [&](int slot) -> bool {
+    bool good = true;
+    if (lane == 0 && f >= (uint32_t)kSlots &&
+        !mbar_wait(&s.slot_empty[slot], ((f / kSlots) - 1) & 1, &s.abort, kTimeoutNs)) {
+      fail(s, p, 0x102);
+      good = false;
+    }
+    return __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+  };
+
   for (int k = blockIdx.x; k < p.n_units && ok; k += gridDim.x) {
     const Unit u = decode(p, k);
+    // lane l tracks sender heads l and l + 32, for the unit's one or two query blocks
+    RowCursor cur[2][2];
+    float wv[2][kAcc];
+#pragma unroll
+    for (int hs = 0; hs < 2; ++hs) {
+      const int sh = lane + 32 * hs;
+      cur[0][hs].start(p, sh, u.I0);
+      cur[1][hs].start(p, sh, p.B == 64 ? u.I1 : -1);
+#pragma unroll
+      for (int g = 0; g < kAcc; ++g) {
+        const int r = u.hg * G + g;
+        wv[hs][g] = (g < G && sh < p.H_s && r < p.H_r) ? __ldg(p.W + (size_t)r * p.H_s + sh) : 0.f;
+      }
+    }
+    bool any_unit = false;
     for (int J = 0; J <= u.Jmax && ok; ++J) {
-      const uint64_t m0 = head_mask(p, u.I0, J);
-      const uint64_t m1 = (p.B == 64) ? head_mask(p, u.I1, J) : m0;
+      bool b[2][2];
+#pragma unroll
+      for (int pt = 0; pt < 2; ++pt)
+#pragma unroll
+        for (int hs = 0; hs < 2; ++hs) {
+          const int I = pt == 0 ? u.I0 : u.I1;
+          b[pt][hs] = (pt == 0 || p.B == 64) && I >= 0 && J <= I ? cur[pt][hs].at(J) : false;
+        }
+      const uint64_t m0 = ((uint64_t)__ballot_sync(0xffffffffu, b[0][1]) << 32) | __ballot_sync(0xffffffffu, b[0][0]);
+      const uint64_t m1 = p.B == 64
+                              ? (((uint64_t)__ballot_sync(0xffffffffu, b[1][1]) << 32) | __ballot_sync(0xffffffffu, b[1][0]))
+                              : m0;
       const uint64_t uni = m0 | m1;
-      if (uni == 0) continue;
-      for (int h = 0; h < nparts && ok; ++h) {
-        const int j0 = J * p.B + 64 * h;
-        // V(n) needs the single V buffer back from the MMAs of sub-step n-1; it is issued as soon
-        // as that is observed, while this sub-step's tiles stream through the ring.
-        bool v_pending = true;
-        uint64_t rem = uni;
-        while (rem != 0 && ok) {
-          const int sh = __ffsll((long long)rem) - 1;
-          rem &= rem - 1;
-          const int slot = (int)(f % kSlots);
-          if (lane == 0 && f >= (uint32_t)kSlots) {
-            if (!mbar_wait(&s.slot_empty[slot], ((f / kSlots) - 1) & 1, &s.abort, kTimeoutNs)) {
-              fail(s, p, 0x102);
+      if (uni != 0) {
+        for (int h = 0; h < nparts && ok; ++h) {
+          const int j0 = J * p.B + 64 * h;
+          bool v_pending = true;
+          uint64_t rem = uni;
+          while (rem != 0 && ok) {
+            const int sh = __ffsll((long long)rem) - 1;
+            rem &= rem - 1;
+            const int slot = (int)(f % kSlots);
+            if (!claim(slot)) {
               ok = false;
+              break;
+            }
+            // tile indices of head sh in both query blocks (kept blocks below J + row start)
+            const int src_lane = sh & 31, hs = sh >> 5;
+            int64_t t[2];
+            float w[kAcc];
+#pragma unroll
+            for (int pt = 0; pt < 2; ++pt) {
+              const int64_t mine0 = cur[pt][0].first + cur[pt][0].count;
+              const int64_t mine1 = cur[pt][1].first + cur[pt][1].count;
+              const int64_t a0 = __shfl_sync(0xffffffffu, mine0, src_lane);
+              const int64_t a1 = __shfl_sync(0xffffffffu, mine1, src_lane);
+              t[pt] = hs ? a1 : a0;
+            }
+#pragma unroll
+            for (int g = 0; g < kAcc; ++g) {
+              const float w0 = __shfl_sync(0xffffffffu, wv[0][g], src_lane);
+              const float w1 = __shfl_sync(0xffffffffu, wv[1][g], src_lane);
+              w[g] = hs ? w1 : w0;
+            }
+            char* dst = reinterpret_cast<char*>(&s.slot[slot][0]);
+            uint32_t bytes = 0, flags = 0;
+            bool zero[2] = {false, false};
+            const char* src[2] = {nullptr, nullptr};
+            const uint32_t len = p.B == 128 ? 16384u : 8192u;
+            for (int pt = 0; pt < (p.B == 64 ? 2 : 1); ++pt) {
+              const uint64_t m = pt == 0 ? m0 : m1;
+              if (!((m >> sh) & 1ull)) continue;
+              flags |= pt == 0 ? kHalf0 : kHalf1;
+              if (t[pt] >= p.capacity) {
+                zero[pt] = true;
+              } else {
+                src[pt] = reinterpret_cast<const char*>(p.vals + t[pt] * (int64_t)p.B * p.B) + (p.B == 128 ? 16384 * h : 0);
+                bytes += len;
+              }
+            }
+            if (p.B == 128) flags |= kHalf1;  // one 128-row panel serves every row
+            for (int pt = 0; pt < 2; ++pt) {
+              if (!zero[pt]) continue;
+              uint4* z = reinterpret_cast<uint4*>(dst + pt * 8192);
+              for (uint32_t e = lane; e < len / 16; e += 32) z[e] = make_uint4(0, 0, 0, 0);
+            }
+            if (rem == 0) flags |= kLastSub;
+            __syncwarp();
+            if (lane == 0) {
+              if (zero[0] || zero[1]) set_status(p.ws, MR_ERR_CAPACITY, 3u);
+#pragma unroll
+              for (int g = 0; g < kAcc; ++g) s.meta[slot].w[g] = w[g];
+              s.meta[slot].flags = flags;
+              mbar_arrive_expect_tx(&s.slot_full[slot], bytes);
+              for (int pt = 0; pt < 2; ++pt)
+                if (src[pt]) bulk_g2s(dst + pt * 8192, src[pt], len, &s.slot_full[slot]);
+              if (v_pending && (nv == 0 || mbar_try_wait(&s.v_empty, (nv - 1) & 1))) {
+                issue_v(u, j0);
+                v_pending = false;
+              }
+            }
+            v_pending = __shfl_sync(0xffffffffu, v_pending ? 1 : 0, 0) != 0;
+            ++f;
+          }
+          if (!ok) break;
+          if (lane == 0 && v_pending) {
+            if (nv > 0 && !mbar_wait(&s.v_empty, (nv - 1) & 1, &s.abort, kTimeoutNs)) {
+              fail(s, p, 0x101);
+              ok = false;
+            } else {
+              issue_v(u, j0);
             }
           }
           ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-          if (!ok) break;
-          char* dst = reinterpret_cast<char*>(&s.slot[slot][0]);
-          // pieces: B=128 -> one 16 KB panel; B=64 -> up to two 8 KB tiles (rows 0-63 / 64-127)
-          uint32_t bytes = 0;
-          bool zero[2] = {false, false};
-          const char* src[2] = {nullptr, nullptr};
-          uint32_t len[2] = {0, 0};
-          for (int part = 0; part < (p.B == 64 ? 2 : 1); ++part) {
-            const int I = part == 0 ? u.I0 : u.I1;
-            const uint64_t m = part == 0 ? m0 : m1;
-            if (!((m >> sh) & 1ull)) continue;
-            const int row = sh * p.nqb + I;
-            const int64_t t = (int64_t)__ldg(p.row_ptr + row) + kept_rank(p.kept_bits + (size_t)row * p.nkw, J);
-            len[part] = p.B == 128 ? 16384u : 8192u;
-            if (t >= p.capacity) {
-              zero[part] = true;
-            } else {
-              src[part] = reinterpret_cast<const char*>(p.vals + t * (int64_t)p.B * p.B) + (p.B == 128 ? 16384 * h : 0);
-              bytes += len[part];
-            }
-          }
-          for (int part = 0; part < 2; ++part) {
-            if (!zero[part]) continue;
-            uint4* z = reinterpret_cast<uint4*>(dst + part * 8192);
-            for (uint32_t e = lane; e < len[part] / 16; e += 32) z[e] = make_uint4(0, 0, 0, 0);
-          }
-          __syncwarp();
-          if (lane == 0) {
-            if (zero[0] || zero[1]) set_status(p.ws, MR_ERR_CAPACITY, 3u);
-            mbar_arrive_expect_tx(&s.slot_full[slot], bytes);
-            for (int part = 0; part < 2; ++part)
-              if (src[part]) bulk_g2s(dst + part * 8192, src[part], len[part], &s.slot_full[slot]);
-            if (v_pending && (nv == 0 || mbar_try_wait(&s.v_empty, (nv - 1) & 1))) {
-              issue_v(u, j0);
-              v_pending = false;
-            }
-          }
-          v_pending = __shfl_sync(0xffffffffu, v_pending ? 1 : 0, 0) != 0;
-          ++f;
+          nv = __shfl_sync(0xffffffffu, nv, 0);
+          any_unit = true;
         }
-        if (!ok) break;
-        if (lane == 0 && v_pending) {
-          if (nv > 0 && !mbar_wait(&s.v_empty, (nv - 1) & 1, &s.abort, kTimeoutNs)) {
-            fail(s, p, 0x101);
-            ok = false;
-          } else {
-            issue_v(u, j0);
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        nv = __shfl_sync(0xffffffffu, nv, 0);
-        if (!ok) break;
       }
+      // advance the kept counts past block J
+#pragma unroll
+      for (int pt = 0; pt < 2; ++pt)
+#pragma unroll
+        for (int hs = 0; hs < 2; ++hs) cur[pt][hs].count += b[pt][hs] ? 1 : 0;
     }
+    if (!ok) break;
+    // mark the end of the unit with a data-less slot (the unit's only slot if it kept nothing)
+    const int slot = (int)(f % kSlots);
+    if (!claim(slot)) {
+      ok = false;
+      break;
+    }
+    if (lane == 0) {
+      s.meta[slot].flags = any_unit ? kLastUnit : (kLastUnit | kEmptyUnit);
+      mbar_arrive(&s.slot_full[slot]);
+    }
+    __syncwarp();
+    ++f;
   }
   // drain: every copy this warp issued must land before the CTA can release its shared memory
   if (lane == 0) {
@@ -226,7 +331,6 @@ __device__ void producer(Smem& s, const Params& p, const CUtensorMap* tmap_v) {
   __syncwarp();
 }
 
-// ------------------------------------------------------------------------------------------------
 template <int G>
 __device__ void mma_issuer(Smem& s, const Params& p) {
   const int lane = threadIdx.x & 31;
@@ -302,10 +406,10 @@ __device__ void mixers(Smem& s, const Params& p) {
   const int row = 32 * (warp & 3) + lane;  // 0..127: this thread's query row within the unit
   const int chalf = warp >> 2;             // which 32 of the sub-step's 64 columns
   const int half = row >> 6;               // for 64-key blocks: which of the two query blocks
+  const uint32_t my_half = half ? kHalf1 : kHalf0;
   const uint32_t row_off = (p.B == 64) ? (uint32_t)(half * 8192 + (row & 63) * 128) : (uint32_t)(row * 128);
   const int sw = row & 7;
   const uint32_t tbase = s.tmem_base;
-  const int nparts = p.B / 64;
   uint32_t f = 0, nsub = 0;
   int nunit = 0;
   bool ok = true;
@@ -313,82 +417,81 @@ __device__ void mixers(Smem& s, const Params& p) {
   for (int k = blockIdx.x; k < p.n_units && ok; k += gridDim.x, ++nunit) {
     const Unit u = decode(p, k);
     bool any = false;
-    for (int J = 0; J <= u.Jmax && ok; ++J) {
-      const uint64_t m0 = head_mask(p, u.I0, J);
-      const uint64_t m1 = (p.B == 64) ? head_mask(p, u.I1, J) : m0;
-      const uint64_t uni = m0 | m1;
-      if (uni == 0) continue;
-      const uint64_t mine = (p.B == 64 && half) ? m1 : m0;
-      for (int h = 0; h < nparts && ok; ++h) {
-        any = true;
+    // sub-steps until the producer's end-of-unit marker slot
+    bool unit_done = false;
+    while (!unit_done && ok) {
 #pragma unroll
-        for (int g = 0; g < G; ++g)
+      for (int g = 0; g < G; ++g)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) acc[g][e] = 0.f;
-        uint64_t rem = uni;
-        while (rem != 0) {
-          const int sh = __ffsll((long long)rem) - 1;
-          rem &= rem - 1;
-          const int slot = (int)(f % kSlots);
-          if (!mbar_wait(&s.slot_full[slot], (f / kSlots) & 1, &s.abort, kTimeoutNs)) {
-            fail(s, p, 0x301);
-            ok = false;
-            break;
-          }
-          if ((mine >> sh) & 1ull) {
-            const char* base = reinterpret_cast<const char*>(&s.slot[slot][0]) + row_off;
-            float w[G];
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-              const int r = u.hg * G + g;
-              w[g] = (r < p.H_r) ? __ldg(p.W + (size_t)r * p.H_s + sh) : 0.f;
-            }
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const uint4 q = *reinterpret_cast<const uint4*>(base + (((4 * chalf + c) ^ sw) << 4));
-              const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float lo = __uint_as_float(wd[e] << 16);
-                const float hi = __uint_as_float(wd[e] & 0xffff0000u);
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                  acc[g][8 * c + 2 * e] = fmaf(w[g], lo, acc[g][8 * c + 2 * e]);
-                  acc[g][8 * c + 2 * e + 1] = fmaf(w[g], hi, acc[g][8 * c + 2 * e + 1]);
-                }
-              }
-            }
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&s.slot_empty[slot]);
-          ++f;
-        }
-        if (!ok) break;
-        // hand X to the tensor core once the previous sub-step's MMAs have read it
-        if (nsub > 0 && !mbar_wait(&s.x_empty, (nsub - 1) & 1, &s.abort, kTimeoutNs)) {
-          fail(s, p, 0x302);
+        for (int e = 0; e < 32; ++e) acc[g][e] = 0.f;
+      bool sub_done = false;
+      while (!sub_done) {
+        const int slot = (int)(f % kSlots);
+        if (!mbar_wait(&s.slot_full[slot], (f / kSlots) & 1, &s.abort, kTimeoutNs)) {
+          fail(s, p, 0x301);
           ok = false;
           break;
         }
+        const uint32_t flags = s.meta[slot].flags;
+        if (flags & kLastUnit) {  // marker slot: no data
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.slot_empty[slot]);
+          ++f;
+          unit_done = true;
+          break;
+        }
+        if (flags & (p.B == 128 ? kHalf1 : my_half)) {
+          const char* base = reinterpret_cast<const char*>(&s.slot[slot][0]) + row_off;
+          float w[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          char* xb = reinterpret_cast<char*>(&s.x[g][0]) + row * 128;
+          for (int g = 0; g < G; ++g) w[g] = s.meta[slot].w[g];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            uint32_t pk[4];
+            const uint4 q = *reinterpret_cast<const uint4*>(base + (((4 * chalf + c) ^ sw) << 4));
+            const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[g][8 * c + 2 * e], acc[g][8 * c + 2 * e + 1]);
-              pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
+              const float lo = __uint_as_float(wd[e] << 16);
+              const float hi = __uint_as_float(wd[e] & 0xffff0000u);
+#pragma unroll
+              for (int g = 0; g < G; ++g) {
+                acc[g][8 * c + 2 * e] = fmaf(w[g], lo, acc[g][8 * c + 2 * e]);
+                acc[g][8 * c + 2 * e + 1] = fmaf(w[g], hi, acc[g][8 * c + 2 * e + 1]);
+              }
             }
-            *reinterpret_cast<uint4*>(xb + (((4 * chalf + c) ^ sw) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         }
-        fence_proxy_async_smem();
+        sub_done = (flags & kLastSub) != 0;
         __syncwarp();
-        if (lane == 0) mbar_arrive(&s.x_full);
-        ++nsub;
+        if (lane == 0) mbar_arrive(&s.slot_empty[slot]);
+        ++f;
       }
+      if (!ok || unit_done) break;
+      any = true;
+      // hand X to the tensor core once the previous sub-step's MMAs have read it
+      if (nsub > 0 && !mbar_wait(&s.x_empty, (nsub - 1) & 1, &s.abort, kTimeoutNs)) {
+        fail(s, p, 0x302);
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        char* xb = reinterpret_cast<char*>(&s.x[g][0]) + row * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[g][8 * c + 2 * e], acc[g][8 * c + 2 * e + 1]);
+            pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          *reinterpret_cast<uint4*>(xb + (((4 * chalf + c) ^ sw) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.x_full);
+      ++nsub;
     }
     if (!ok) break;
     // ---- epilogue: accumulators -> bf16 -> O ----

@@ -517,6 +517,20 @@ cudaError_t compress_impl(const CompressArgs& a) {
   return cudaGetLastError();
 }
 
+template <typename T, typename TV, int BLK, int D>
+cudaError_t emit_impl(const CompressArgs& a) {
+  const int nqb = a.L / BLK;
+  const size_t smem = (size_t)2 * BLK * (D + 1) * sizeof(float);
+  auto k3 = k_emit<T, TV, BLK, D>;
+  cudaError_t e = set_smem(k3, smem);
+  if (e != cudaSuccess) return e;
+  ProfScope ps(kKEmit, a.stream);
+  k3<<<a.H * nqb, kThreads, smem, a.stream>>>(
+      (const T*)a.Q, (const T*)a.K, a.H, a.L, a.scale, a.bias, a.lse_ws, a.map.row_ptr,
+      a.map.kept_bits, a.map.capacity_tiles, a.map.col_idx, (TV*)a.map.vals);
+  return cudaGetLastError();
+}
+
 template <typename T, int BLK, int DV>
 cudaError_t retrieve_impl(const RetrieveArgs& a) {
   const int nqb = a.map.L / BLK;
@@ -561,6 +575,15 @@ cudaError_t simt_compress(const CompressArgs& a) {
   if (a.block == 64 && a.d == 128) return bf ? compress_impl<__nv_bfloat16, __nv_bfloat16, 64, 128>(a) : compress_impl<float, float, 64, 128>(a);
   if (a.block == 128 && a.d == 64) return bf ? compress_impl<__nv_bfloat16, __nv_bfloat16, 128, 64>(a) : compress_impl<float, float, 128, 64>(a);
   if (a.block == 128 && a.d == 128) return bf ? compress_impl<__nv_bfloat16, __nv_bfloat16, 128, 128>(a) : compress_impl<float, float, 128, 128>(a);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t simt_emit(const CompressArgs& a) {
+  const bool bf = a.dt == MR_BF16;
+  if (a.block == 64 && a.d == 64) return bf ? emit_impl<__nv_bfloat16, __nv_bfloat16, 64, 64>(a) : emit_impl<float, float, 64, 64>(a);
+  if (a.block == 64 && a.d == 128) return bf ? emit_impl<__nv_bfloat16, __nv_bfloat16, 64, 128>(a) : emit_impl<float, float, 64, 128>(a);
+  if (a.block == 128 && a.d == 64) return bf ? emit_impl<__nv_bfloat16, __nv_bfloat16, 128, 64>(a) : emit_impl<float, float, 128, 64>(a);
+  if (a.block == 128 && a.d == 128) return bf ? emit_impl<__nv_bfloat16, __nv_bfloat16, 128, 128>(a) : emit_impl<float, float, 128, 128>(a);
   return cudaErrorInvalidValue;
 }
 
