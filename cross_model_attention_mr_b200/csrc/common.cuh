@@ -56,6 +56,19 @@ __device__ __forceinline__ float bias_term(const Bias& b, int h, int i, int j) {
   return best == -INFINITY ? 0.f : best;
 }
 
+// The same rule split for tile kernels: the key-block term kb (already looked up for a chunk of
+// keys inside one key block, -inf = none) combined with the sink and window terms of (i, j).
+__device__ __forceinline__ float bias_with_kb(const Bias& b, int i, int j, float kb) {
+  float best = kb;
+  if (j < b.sink_len) best = fmaxf(best, b.sink_bias);
+  if (i - j < b.window) best = fmaxf(best, b.window_bias);
+  return best == -INFINITY ? 0.f : best;
+}
+
+__device__ __forceinline__ float kb_term(const Bias& b, int h, int j) {
+  return b.kb == nullptr ? -INFINITY : __ldg(b.kb + (size_t)h * b.n_kb + j / b.kb_block);
+}
+
 template <typename T>
 __device__ __forceinline__ float to_f32(T x);
 template <>

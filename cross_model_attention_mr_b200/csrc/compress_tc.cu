@@ -171,11 +171,26 @@ __device__ void mma_issuer(Smem& s, const Params& p) {
 // ------------------------------------------------------------------------------------------------
 // Softmax warpgroups
 // ------------------------------------------------------------------------------------------------
+// Maximum of 32 values as a tree (short dependency chains).
 __device__ __forceinline__ float warp_max32(const float (&v)[32]) {
-  float m = v[0];
+  float m[16];
 #pragma unroll
-  for (int t = 1; t < 32; ++t) m = fmaxf(m, v[t]);
-  return m;
+  for (int t = 0; t < 16; ++t) m[t] = fmaxf(v[t], v[t + 16]);
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+    for (int t = 0; t < w; ++t) m[t] = fmaxf(m[t], m[t + w]);
+  return m[0];
+}
+
+// Sum of 2^x over 32 values with 8 independent partial sums.
+__device__ __forceinline__ float sum_ex2_32(const float (&x)[32]) {
+  float a[8];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) a[t] = ex2_approx(x[t]);
+#pragma unroll
+  for (int t = 8; t < 32; ++t) a[t & 7] += ex2_approx(x[t]);
+  return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
 
 // Base-2 bias offset of key j for head h when only the key-block term can apply.
@@ -220,65 +235,77 @@ __device__ void softmax_group(Smem& s, const Params& p, int w) {
       float acc[2] = {0.f, 0.f};
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
-        uint32_t raw[2][32];
-        tmem_ld32(tbase + lane_addr + 128 * w + 64 * hh, raw[0]);
-        tmem_ld32(tbase + lane_addr + 128 * w + 64 * hh + 32, raw[1]);
-        tmem_wait_ld();
+        // 64 logits of this row: keys j_tile + 64 hh .. + 63 (one key block when the block is 64)
+        float v[2][32];
+        {
+          uint32_t raw[2][32];
+          tmem_ld32(tbase + lane_addr + 128 * w + 64 * hh, raw[0]);
+          tmem_ld32(tbase + lane_addr + 128 * w + 64 * hh + 32, raw[1]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+            for (int t = 0; t < 32; ++t) v[cc][t] = __uint_as_float(raw[cc][t]);
+        }
         if (hh == 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&s.s_empty[w]);
         }
+        const int j0 = j_tile + 64 * hh;
+        float off[2] = {0.f, 0.f};
+        float mc;
+        if (!special) {
+          // only the key-block term can apply: a constant per 32 keys
+          off[0] = kb_offset(p.bias, h, j0);
+          off[1] = kb_offset(p.bias, h, j0 + 32);
+          mc = fmaxf(fmaf(warp_max32(v[0]), p.a, off[0]), fmaf(warp_max32(v[1]), p.a, off[1]));
+        } else {
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int chunk = 2 * hh + cc;
-          const int j0 = j_tile + 32 * chunk;
-          float v[32];
-          float mc, off = 0.f;
-          if (!special) {
-            off = kb_offset(p.bias, h, j0);
-#pragma unroll
-            for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(raw[cc][t]);
-            mc = fmaf(warp_max32(v), p.a, off);
-          } else {
+          for (int cc = 0; cc < 2; ++cc) {
+            const float kb = kb_term(p.bias, h, j0 + 32 * cc);
 #pragma unroll
             for (int t = 0; t < 32; ++t) {
-              const int j = j0 + t;
-              v[t] = (row_ok && j <= i) ? fmaf(__uint_as_float(raw[cc][t]), p.a, bias_term(p.bias, h, i, j) * kLog2e)
-                                        : -INFINITY;
+              const int j = j0 + 32 * cc + t;
+              v[cc][t] = (row_ok && j <= i) ? fmaf(v[cc][t], p.a, bias_with_kb(p.bias, i, j, kb) * kLog2e) : -INFINITY;
             }
-            mc = warp_max32(v);
           }
-          if (!row_ok) mc = -INFINITY;
-          const bool need = mc > c + kRescale;
-          if (__any_sync(0xffffffffu, need)) {
-            const float cn = need ? mc : c;
-            const float f = need ? ex2_approx(c - cn) : 1.f;  // c = -inf gives 0
-            acc[0] *= f;
-            acc[1] *= f;
-            for (int c0 = 0; c0 < used; c0 += 32) {
-              uint32_t xs[32];
-              tmem_ld32(tbase + lane_addr + xbase + c0, xs);
-              tmem_wait_ld();
-#pragma unroll
-              for (int t = 0; t < 32; ++t) xs[t] = __float_as_uint(__uint_as_float(xs[t]) * f);
-              tmem_st32(tbase + lane_addr + xbase + c0, xs);
-            }
-            tmem_wait_st();
-            c = cn;
-          }
-          const int kb = (p.B == 64 && chunk >= 2) ? 1 : 0;
-          float sum = 0.f;
-          if (!special) {
-            const float o = off - c;
-#pragma unroll
-            for (int t = 0; t < 32; ++t) sum += ex2_approx(fmaf(v[t], p.a, o));
-          } else if (c != -INFINITY) {
-#pragma unroll
-            for (int t = 0; t < 32; ++t) sum += ex2_approx(v[t] - c);  // -inf gives 0
-          }
-          acc[kb] += row_ok ? sum : 0.f;
+          mc = fmaxf(warp_max32(v[0]), warp_max32(v[1]));
         }
+        if (!row_ok) mc = -INFINITY;
+        const bool need = mc > c + kRescale;
+        if (__any_sync(0xffffffffu, need)) {
+          const float cn = need ? mc : c;
+          const float f = need ? ex2_approx(c - cn) : 1.f;  // c = -inf gives 0
+          acc[0] *= f;
+          acc[1] *= f;
+          for (int c0 = 0; c0 < used; c0 += 32) {
+            uint32_t xs[32];
+            tmem_ld32(tbase + lane_addr + xbase + c0, xs);
+            tmem_wait_ld();
+#pragma unroll
+            for (int t = 0; t < 32; ++t) xs[t] = __float_as_uint(__uint_as_float(xs[t]) * f);
+            tmem_st32(tbase + lane_addr + xbase + c0, xs);
+          }
+          tmem_wait_st();
+          c = cn;
+        }
+        float sum = 0.f;
+        if (c != -INFINITY && row_ok) {
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            if (!special) {
+              const float o = off[cc] - c;
+#pragma unroll
+              for (int t = 0; t < 32; ++t) v[cc][t] = fmaf(v[cc][t], p.a, o);
+            } else {
+#pragma unroll
+              for (int t = 0; t < 32; ++t) v[cc][t] -= c;  // -inf stays -inf and gives 0
+            }
+            sum += sum_ex2_32(v[cc]);
+          }
+        }
+        acc[(p.B == 64) ? hh : 0] += sum;
       }
       if (per_tile == 1)
         tmem_st1(tbase + lane_addr + xbase + used, __float_as_uint(acc[0]));

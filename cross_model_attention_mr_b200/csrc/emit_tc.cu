@@ -48,14 +48,13 @@ struct Params {
 struct Smem {
   __nv_bfloat16 q[2][128 * 64];
   __nv_bfloat16 k[kKStages][2][128 * 64];
-  __nv_bfloat16 stage[2][128 * 128];  // per warpgroup: one tile in storage order
+  __nv_bfloat16 stage[2][128 * 128];  // per warpgroup: 4 warps x (2 key halves x 32 rows x 128 B)
   uint64_t q_full, q_empty;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t s_full[2], s_empty[2];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
-  int wg_fail[2];  // written by a warpgroup's warps only before a barrier, read after it
 };
 
 __device__ __forceinline__ void fail(Smem& s, const Params& p, uint32_t detail) {
@@ -68,21 +67,74 @@ __device__ __forceinline__ void unit_of(const Params& p, int k, int& h, int& rb)
   h = k % p.H;
 }
 
-__device__ __forceinline__ bool kept(const Params& p, int h, int I, int J) {
-  if (I < 0 || I >= p.nqb || J > I) return false;
-  return (__ldg(p.kept_bits + (size_t)(h * p.nqb + I) * p.nkw + (J >> 5)) >> (J & 31)) & 1u;
-}
+// One query block's kept bits, walked with non-decreasing J: kept flag, and the BSR position of
+// each kept tile (row start + kept blocks so far).
+struct QCursor {
+  const uint32_t* bits;
+  uint32_t word;
+  int word_idx, count, I;
+  int64_t first;
+  bool live;
+  __device__ __forceinline__ void start(const Params& p, int h, int I_) {
+    I = I_;
+    live = I_ >= 0 && I_ < p.nqb;
+    count = 0;
+    word_idx = 0;
+    word = 0u;
+    first = 0;
+    bits = nullptr;
+    if (live) {
+      const int u = h * p.nqb + I_;
+      bits = p.kept_bits + (size_t)u * p.nkw;
+      word = __ldg(bits);
+      first = __ldg(p.row_ptr + u);
+    }
+  }
+  __device__ __forceinline__ bool kept(int J) {
+    if (!live || J > I) return false;
+    const int wi = J >> 5;
+    if (wi != word_idx) {
+      word_idx = wi;
+      word = __ldg(bits + wi);
+    }
+    return (word >> (J & 31)) & 1u;
+  }
+};
 
-// Which 64 x 64 (B = 64) or 128 x 128 (B = 128) pieces of key tile T the unit emits:
-// bit (2 * rowhalf + colhalf) for B = 64, bit 0 for B = 128.
-__device__ __forceinline__ uint32_t tile_pieces(const Params& p, int h, int rb, int T) {
-  if (p.B == 128) return kept(p, h, rb, T) ? 1u : 0u;
-  uint32_t m = 0;
-  for (int rh = 0; rh < 2; ++rh)
-    for (int ch = 0; ch < 2; ++ch)
-      if (kept(p, h, 2 * rb + rh, 2 * T + ch)) m |= 1u << (2 * rh + ch);
-  return m;
-}
+// The unit's one (block 128) or two (block 64) query blocks.  pieces(T) returns which pieces of
+// key tile T are stored -- bit (2 * row half + key half) for block 64, bit 0 for block 128 -- with
+// their BSR positions, and must be called for every T in increasing order.
+struct UnitCursor {
+  QCursor q[2];
+  __device__ __forceinline__ void start(const Params& p, int h, int rb) {
+    if (p.B == 128) {
+      q[0].start(p, h, rb);
+      q[1].start(p, h, -1);
+    } else {
+      q[0].start(p, h, 2 * rb);
+      q[1].start(p, h, 2 * rb + 1);
+    }
+  }
+  __device__ __forceinline__ uint32_t pieces(const Params& p, int T, int64_t (&t)[4]) {
+    uint32_t m = 0;
+    if (p.B == 128) {
+      if (q[0].kept(T)) {
+        m = 1u;
+        t[0] = q[0].first + q[0].count++;
+      }
+      return m;
+    }
+#pragma unroll
+    for (int rh = 0; rh < 2; ++rh)
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch)
+        if (q[rh].kept(2 * T + ch)) {
+          m |= 1u << (2 * rh + ch);
+          t[2 * rh + ch] = q[rh].first + q[rh].count++;
+        }
+    return m;
+  }
+};
 
 __device__ void producer(Smem& s, const Params& p, const CUtensorMap* tq, const CUtensorMap* tk) {
   if ((threadIdx.x & 31) != 0) return;
@@ -99,8 +151,11 @@ __device__ void producer(Smem& s, const Params& p, const CUtensorMap* tq, const 
     mbar_arrive_expect_tx(&s.q_full, 2 * 128 * 64 * 2);
     tma_load_2d(&s.q[0][0], tq, &s.q_full, 0, qrow);
     tma_load_2d(&s.q[1][0], tq, &s.q_full, 64, qrow);
+    UnitCursor uc;
+    uc.start(p, h, rb);
     for (int T = 0; T <= rb; ++T) {
-      if (!tile_pieces(p, h, rb, T)) continue;
+      int64_t tpos[4];
+      if (!uc.pieces(p, T, tpos)) continue;
       const int st = (int)(nk % kKStages);
       if (nk >= (uint32_t)kKStages && !mbar_wait(&s.k_empty[st], ((nk / kKStages) - 1) & 1, &s.abort, kTimeoutNs)) {
         fail(s, p, 0x502);
@@ -134,8 +189,11 @@ __device__ void mma_issuer(Smem& s, const Params& p) {
       break;
     }
     int n_local = 0;
+    UnitCursor uc;
+    uc.start(p, h, rb);
     for (int T = 0; T <= rb; ++T) {
-      if (!tile_pieces(p, h, rb, T)) continue;
+      int64_t tpos[4];
+      if (!uc.pieces(p, T, tpos)) continue;
       const int st = (int)(nk % kKStages), b = n_local & 1;
       if (!mbar_wait(&s.k_full[st], (nk / kKStages) & 1, &s.abort, kTimeoutNs) ||
           (nb[b] > 0 && !mbar_wait(&s.s_empty[b], (nb[b] - 1) & 1, &s.abort, kTimeoutNs))) {
@@ -171,49 +229,54 @@ __device__ __forceinline__ float kb_offset(const Bias& b, int h, int j) {
   return v == -INFINITY ? 0.f : v * kLog2e;
 }
 
+// One warpgroup: each warp handles 32 query rows of every tile given to the warpgroup, stages
+// them in the map's storage order and stores them with its own bulk copies (the 32 rows of a
+// panel are contiguous in the stored tile), so the warps of the group never wait on each other.
 __device__ void emit_group(Smem& s, const Params& p, int w) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q4 = warp & 3;
   const int row = 32 * q4 + lane;
-  const int gtid = threadIdx.x - 32 * (kSoftmaxWarp0 + 4 * w);
   const uint32_t tbase = s.tmem_base;
   const uint32_t lane_addr = (uint32_t)(32 * q4) << 16;
-  const uint32_t bar_id = 2 + w;
-  char* stage = reinterpret_cast<char*>(&s.stage[w][0]);
+  char* stage = reinterpret_cast<char*>(&s.stage[w][0]) + 8192 * q4;  // 2 x 4 KB: key halves
+  const int rh = row >> 6;  // block 64: which query block of the unit this warp's rows belong to
   uint32_t nb = 0;
-  bool ok = true;
   bool store_pending = false;
+  bool ok = true;
   for (int k = blockIdx.x; k < p.n_units && ok; k += gridDim.x) {
     int h, rb;
     unit_of(p, k, h, rb);
     const int i = 128 * rb + row;
     const bool row_ok = i < p.L;
     const float lse2 = row_ok ? __ldg(p.lse_ws + (size_t)h * p.L + i) * kLog2e : 0.f;
-    const int rh = row >> 6;  // B = 64: which query block of the unit this row belongs to
+    UnitCursor uc;
+    uc.start(p, h, rb);
     int n_local = 0;
-    for (int T = 0; T <= rb && ok; ++T) {
-      const uint32_t pieces = tile_pieces(p, h, rb, T);
+    for (int T = 0; T <= rb; ++T) {
+      int64_t tpos[4];
+      const uint32_t pieces = uc.pieces(p, T, tpos);
       if (!pieces) continue;
       const int mine = n_local++ & 1;
       if (mine != w) continue;
       if (!mbar_wait(&s.s_full[w], nb & 1, &s.abort, kTimeoutNs)) {
         fail(s, p, 0x521);
-        s.wg_fail[w] = 1;
+        ok = false;
+        break;
       }
       ++nb;
       tc_fence_after();
-      // the staging buffer may still be read by this warpgroup's previous bulk store
-      if (gtid == 0 && store_pending) bulk_wait_read<0>();
-      named_sync(bar_id, 128);
-      // every warp of the warpgroup takes the same decision and passes the same barriers
-      const bool stop = s.wg_fail[w] != 0;
+      // the staging buffer may still be read by this warp's previous bulk stores
+      if (store_pending) {
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+      }
       const int j_tile = 128 * T;
       const bool special = (T == rb) || (j_tile < p.bias.sink_len) ||
                            (p.bias.window > 0 && j_tile + 127 > 128 * rb - p.bias.window);
-      // which 64-key halves of this row's tile are stored
+      // which 64-key halves of this warp's rows are stored
       const uint32_t row_mask = p.B == 128 ? 3u : ((pieces >> (2 * rh)) & 3u);
 #pragma unroll
-      for (int hh = 0; hh < 2 && !stop; ++hh) {
+      for (int hh = 0; hh < 2; ++hh) {
         uint32_t raw[2][32];
         tmem_ld32(tbase + lane_addr + 128 * w + 64 * hh, raw[0]);
         tmem_ld32(tbase + lane_addr + 128 * w + 64 * hh + 32, raw[1]);
@@ -224,8 +287,7 @@ __device__ void emit_group(Smem& s, const Params& p, int w) {
           if (lane == 0) mbar_arrive(&s.s_empty[w]);
         }
         if (!((row_mask >> hh) & 1u)) continue;  // warp-uniform
-        // destination: panel hh (B = 128) or the 64 x 64 piece (rh, hh) (B = 64)
-        char* dst = p.B == 128 ? stage + 16384 * hh + row * 128 : stage + 8192 * (2 * rh + hh) + (row & 63) * 128;
+        char* dst = stage + 4096 * hh + lane * 128;
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int j0 = j_tile + 64 * hh + 32 * cc;
@@ -235,11 +297,12 @@ __device__ void emit_group(Smem& s, const Params& p, int w) {
 #pragma unroll
             for (int t = 0; t < 32; ++t) pr[t] = ex2_approx(fmaf(__uint_as_float(raw[cc][t]), p.a, o));
           } else {
+            const float kb = kb_term(p.bias, h, j0);
 #pragma unroll
             for (int t = 0; t < 32; ++t) {
               const int j = j0 + t;
               pr[t] = (row_ok && j <= i)
-                          ? ex2_approx(fmaf(__uint_as_float(raw[cc][t]), p.a, bias_term(p.bias, h, i, j) * kLog2e) - lse2)
+                          ? ex2_approx(fmaf(__uint_as_float(raw[cc][t]), p.a, bias_with_kb(p.bias, i, j, kb) * kLog2e) - lse2)
                           : 0.f;
             }
           }
@@ -252,36 +315,38 @@ __device__ void emit_group(Smem& s, const Params& p, int w) {
               pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
             }
             const int chunk = 4 * cc + c8;  // 16-byte chunk within the 64-column panel row
-            *reinterpret_cast<uint4*>(dst + ((chunk ^ (row & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(dst + ((chunk ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         }
       }
       fence_proxy_async_smem();
-      named_sync(bar_id, 128);
-      if (stop) {
-        ok = false;
-        break;
-      }
-      if (gtid == 0) {
-        // one bulk store per stored tile (B = 128) or 64 x 64 piece (B = 64)
-        for (int piece = 0; piece < (p.B == 128 ? 1 : 4); ++piece) {
-          if (!((pieces >> piece) & 1u)) continue;
-          const int I = p.B == 128 ? rb : 2 * rb + (piece >> 1);
-          const int J = p.B == 128 ? T : 2 * T + (piece & 1);
-          const int u = h * p.nqb + I;
-          const int64_t t = (int64_t)__ldg(p.row_ptr + u) + kept_rank(p.kept_bits + (size_t)u * p.nkw, J);
+      __syncwarp();
+      if (lane == 0) {
+        bool issued = false;
+        for (int hh = 0; hh < 2; ++hh) {
+          if (!((row_mask >> hh) & 1u)) continue;
+          const int piece = p.B == 128 ? 0 : 2 * rh + hh;
+          const int64_t t = tpos[piece];
           if (t >= p.capacity) continue;
+          // destination: panel hh of the 128-tile, or the (rh, hh) 64-tile; this warp's 32 rows
           const int64_t tbytes = (int64_t)p.B * p.B * 2;
-          bulk_s2g(reinterpret_cast<char*>(p.vals) + t * tbytes, stage + (p.B == 128 ? 0 : 8192 * piece),
-                   (uint32_t)tbytes);
-          p.col_idx[t] = J;
+          char* gdst = reinterpret_cast<char*>(p.vals) + t * tbytes +
+                       (p.B == 128 ? 16384 * hh + 4096 * q4 : 4096 * (q4 & 1));
+          bulk_s2g(gdst, stage + 4096 * hh, 4096);
+          issued = true;
+          const bool writer = p.B == 128 ? (q4 == 0 && hh == 0) : ((q4 & 1) == 0);
+          if (writer) p.col_idx[t] = p.B == 128 ? T : 2 * T + hh;
         }
-        bulk_commit();
-        store_pending = true;
+        if (issued) {
+          bulk_commit();
+          store_pending = true;
+        }
       }
+      store_pending = __shfl_sync(0xffffffffu, store_pending ? 1 : 0, 0) != 0;
     }
   }
-  if (gtid == 0 && store_pending) bulk_wait_all<0>();
+  if (lane == 0 && store_pending) bulk_wait_all<0>();
+  __syncwarp();
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -302,7 +367,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&s.mma_done, 1);
     s.abort = 0;
-    s.wg_fail[0] = s.wg_fail[1] = 0;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {

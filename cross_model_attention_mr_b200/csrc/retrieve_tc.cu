@@ -31,10 +31,11 @@ namespace {
 using namespace sm100;
 
 constexpr int kMixWarps = 8;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kThreads = 320;
-constexpr int kSlots = 5;
+constexpr int kProducerWarp0 = 8;  // producer warps 8, 9, 10 (each owns ring slots p and p + 3)
+constexpr int kProducers = 3;
+constexpr int kMmaWarp = 11;
+constexpr int kThreads = 384;
+constexpr int kSlots = 6;
 constexpr int kSlotBytes = 16384;
 constexpr int kAcc = 4;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
@@ -150,11 +151,16 @@ struct RowCursor {
   }
 };
 
+// Producer warp `pw` (0..2).  Bulk copies are issued by several warps because one issuing warp
+// is limited to a few million copies per second; each warp fills only the ring slots it owns
+// (slot % 3 == pw), so a slot's fills are always issued by one warp, in order, each after the
+// release of the previous one.  All producer warps walk the same unit / key-block sequence.
 template <int G>
-__device__ void producer(Smem& s, const Params& p, const CUtensorMap* tmap_v) {
+__device__ void producer(Smem& s, const Params& p, const CUtensorMap* tmap_v, int pw) {
   const int lane = threadIdx.x & 31;
-  uint32_t f = 0;   // slot fills issued
-  uint32_t nv = 0;  // V fills issued (one per executed sub-step)
+  uint32_t f = 0;   // slot fills in the sequence so far (all warps)
+  uint32_t nv = 0;  // V fills issued (warp 0 only; one per executed sub-step)
+  uint32_t hi = 0;  // one past the last fill this warp issued
   const int nparts = p.B / 64;
   bool ok = true;
 
@@ -173,12 +179,12 @@ __device__ void producer(Smem& s, const Params& p, const CUtensorMap* tmap_v) {
     }
     ++nv;
   };
-
-  // claim the next ring slot (lane 0 waits), returns false on timeout
-  auto claim = [&](int slot) -> bool {
+  auto owns = [&](uint32_t F) { return (int)((F % kSlots) % kProducers) == pw; };
+  // lane 0 waits until the slot of fill F is free (its previous fill, issued by this warp, released)
+  auto claim = [&](uint32_t F) -> bool {
     bool good = true;
-    if (lane == 0 && f >= (uint32_t)kSlots &&
-        !mbar_wait(&s.slot_empty[slot], ((f / kSlots) - 1) & 1, &s.abort, kTimeoutNs)) {
+    if (lane == 0 && F >= (uint32_t)kSlots &&
+        !mbar_wait(&s.slot_empty[F % kSlots], ((F / kSlots) - 1) & 1, &s.abort, kTimeoutNs)) {
       fail(s, p, 0x102);
       good = false;
     }
@@ -217,78 +223,71 @@ __device__ void producer(Smem& s, const Params& p, const CUtensorMap* tmap_v) {
                               : m0;
       const uint64_t uni = m0 | m1;
       if (uni != 0) {
+        const int nsl = __popcll((long long)uni);
         for (int h = 0; h < nparts && ok; ++h) {
           const int j0 = J * p.B + 64 * h;
-          bool v_pending = true;
           uint64_t rem = uni;
-          while (rem != 0 && ok) {
+          for (int rank = 0; rank < nsl && ok; ++rank) {
             const int sh = __ffsll((long long)rem) - 1;
             rem &= rem - 1;
-            const int slot = (int)(f % kSlots);
-            if (!claim(slot)) {
+            const uint32_t F = f + (uint32_t)rank;
+            if (!owns(F)) continue;  // warp-uniform
+            if (!claim(F)) {
               ok = false;
               break;
             }
-            // tile indices of head sh in both query blocks (kept blocks below J + row start)
             const int src_lane = sh & 31, hs = sh >> 5;
             int64_t t[2];
-            float w[kAcc];
+            bool use[2];
 #pragma unroll
             for (int pt = 0; pt < 2; ++pt) {
-              const int64_t mine0 = cur[pt][0].first + cur[pt][0].count;
-              const int64_t mine1 = cur[pt][1].first + cur[pt][1].count;
-              const int64_t a0 = __shfl_sync(0xffffffffu, mine0, src_lane);
-              const int64_t a1 = __shfl_sync(0xffffffffu, mine1, src_lane);
-              t[pt] = hs ? a1 : a0;
+              const int64_t t0 = __shfl_sync(0xffffffffu, cur[pt][0].first + cur[pt][0].count, src_lane);
+              const int64_t t1 = __shfl_sync(0xffffffffu, cur[pt][1].first + cur[pt][1].count, src_lane);
+              t[pt] = hs ? t1 : t0;
+              use[pt] = ((pt == 0 ? m0 : m1) >> sh) & 1ull;
             }
+            float w[kAcc];
 #pragma unroll
             for (int g = 0; g < kAcc; ++g) {
               const float w0 = __shfl_sync(0xffffffffu, wv[0][g], src_lane);
               const float w1 = __shfl_sync(0xffffffffu, wv[1][g], src_lane);
               w[g] = hs ? w1 : w0;
             }
-            char* dst = reinterpret_cast<char*>(&s.slot[slot][0]);
-            uint32_t bytes = 0, flags = 0;
-            bool zero[2] = {false, false};
-            const char* src[2] = {nullptr, nullptr};
-            const uint32_t len = p.B == 128 ? 16384u : 8192u;
-            for (int pt = 0; pt < (p.B == 64 ? 2 : 1); ++pt) {
-              const uint64_t m = pt == 0 ? m0 : m1;
-              if (!((m >> sh) & 1ull)) continue;
-              flags |= pt == 0 ? kHalf0 : kHalf1;
-              if (t[pt] >= p.capacity) {
-                zero[pt] = true;
-              } else {
-                src[pt] = reinterpret_cast<const char*>(p.vals + t[pt] * (int64_t)p.B * p.B) + (p.B == 128 ? 16384 * h : 0);
-                bytes += len;
-              }
-            }
-            if (p.B == 128) flags |= kHalf1;  // one 128-row panel serves every row
-            for (int pt = 0; pt < 2; ++pt) {
-              if (!zero[pt]) continue;
-              uint4* z = reinterpret_cast<uint4*>(dst + pt * 8192);
-              for (uint32_t e = lane; e < len / 16; e += 32) z[e] = make_uint4(0, 0, 0, 0);
-            }
-            if (rem == 0) flags |= kLastSub;
-            __syncwarp();
             if (lane == 0) {
-              if (zero[0] || zero[1]) set_status(p.ws, MR_ERR_CAPACITY, 3u);
+              const int slot = (int)(F % kSlots);
+              char* dst = reinterpret_cast<char*>(&s.slot[slot][0]);
+              uint32_t bytes = 0, flags = 0;
+              const uint32_t len = p.B == 128 ? 16384u : 8192u;
+              const char* src[2] = {nullptr, nullptr};
+              for (int pt = 0; pt < (p.B == 64 ? 2 : 1); ++pt) {
+                if (!use[pt]) continue;
+                flags |= pt == 0 ? kHalf0 : kHalf1;
+                if (t[pt] >= p.capacity) {
+                  // the map overflowed: this tile was never stored; contribute zeros
+                  uint4* z = reinterpret_cast<uint4*>(dst + pt * 8192);
+                  for (uint32_t e = 0; e < len / 16; ++e) z[e] = make_uint4(0, 0, 0, 0);
+                  set_status(p.ws, MR_ERR_CAPACITY, 3u);
+                } else {
+                  src[pt] = reinterpret_cast<const char*>(p.vals + t[pt] * (int64_t)p.B * p.B) + (p.B == 128 ? 16384 * h : 0);
+                  bytes += len;
+                }
+              }
+              if (p.B == 128) flags |= kHalf1;  // one 128-row panel serves every row
+              if (rank == nsl - 1) flags |= kLastSub;
 #pragma unroll
               for (int g = 0; g < kAcc; ++g) s.meta[slot].w[g] = w[g];
               s.meta[slot].flags = flags;
               mbar_arrive_expect_tx(&s.slot_full[slot], bytes);
               for (int pt = 0; pt < 2; ++pt)
                 if (src[pt]) bulk_g2s(dst + pt * 8192, src[pt], len, &s.slot_full[slot]);
-              if (v_pending && (nv == 0 || mbar_try_wait(&s.v_empty, (nv - 1) & 1))) {
-                issue_v(u, j0);
-                v_pending = false;
-              }
             }
-            v_pending = __shfl_sync(0xffffffffu, v_pending ? 1 : 0, 0) != 0;
-            ++f;
+            hi = F + 1;
+            __syncwarp();
           }
           if (!ok) break;
-          if (lane == 0 && v_pending) {
+          f += (uint32_t)nsl;
+          // V of this sub-step (warp 0), once the previous sub-step's MMAs released the V buffer
+          if (pw == 0 && lane == 0) {
             if (nv > 0 && !mbar_wait(&s.v_empty, (nv - 1) & 1, &s.abort, kTimeoutNs)) {
               fail(s, p, 0x101);
               ok = false;
@@ -309,23 +308,25 @@ __device__ void producer(Smem& s, const Params& p, const CUtensorMap* tmap_v) {
     }
     if (!ok) break;
     // mark the end of the unit with a data-less slot (the unit's only slot if it kept nothing)
-    const int slot = (int)(f % kSlots);
-    if (!claim(slot)) {
-      ok = false;
-      break;
+    if (owns(f)) {
+      if (!claim(f)) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) {
+        s.meta[f % kSlots].flags = any_unit ? kLastUnit : (kLastUnit | kEmptyUnit);
+        mbar_arrive(&s.slot_full[f % kSlots]);
+      }
+      hi = f + 1;
+      __syncwarp();
     }
-    if (lane == 0) {
-      s.meta[slot].flags = any_unit ? kLastUnit : (kLastUnit | kEmptyUnit);
-      mbar_arrive(&s.slot_full[slot]);
-    }
-    __syncwarp();
     ++f;
   }
   // drain: every copy this warp issued must land before the CTA can release its shared memory
   if (lane == 0) {
     const int never = 0;  // drain even after an abort: wait on the copies themselves (bounded)
-    for (uint32_t g = (f > (uint32_t)kSlots ? f - kSlots : 0); g < f; ++g)
-      mbar_wait(&s.slot_full[g % kSlots], (g / kSlots) & 1, &never, kTimeoutNs);
+    for (uint32_t g = (hi > (uint32_t)kSlots ? hi - kSlots : 0); g < hi; ++g)
+      if (owns(g)) mbar_wait(&s.slot_full[g % kSlots], (g / kSlots) & 1, &never, kTimeoutNs);
     if (nv > 0) mbar_wait(&s.v_full, (nv - 1) & 1, &never, kTimeoutNs);
   }
   __syncwarp();
@@ -400,71 +401,86 @@ __device__ void mma_issuer(Smem& s, const Params& p) {
 }
 
 // ------------------------------------------------------------------------------------------------
+// What a mixer thread takes from one ring slot: the slot's flags and weights and its own 32
+// columns of its own row (4 x 16 bytes).
+struct SlotData {
+  uint32_t flags;
+  float w[kAcc];
+  uint4 d[4];
+};
+
 template <int G>
 __device__ void mixers(Smem& s, const Params& p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = 32 * (warp & 3) + lane;  // 0..127: this thread's query row within the unit
   const int chalf = warp >> 2;             // which 32 of the sub-step's 64 columns
   const int half = row >> 6;               // for 64-key blocks: which of the two query blocks
-  const uint32_t my_half = half ? kHalf1 : kHalf0;
+  const uint32_t use_mask = (p.B == 128) ? kHalf1 : (half ? kHalf1 : kHalf0);
   const uint32_t row_off = (p.B == 64) ? (uint32_t)(half * 8192 + (row & 63) * 128) : (uint32_t)(row * 128);
   const int sw = row & 7;
   const uint32_t tbase = s.tmem_base;
-  uint32_t f = 0, nsub = 0;
+  uint32_t fetched = 0, nsub = 0;
   int nunit = 0;
   bool ok = true;
-  float acc[G][32];
+
+  // Wait for the next fill, copy what this thread needs into registers, and hand the slot back
+  // to the producer at once (the arrive orders the reads before any refill).
+  auto fetch = [&](SlotData& o) -> bool {
+    const int slot = (int)(fetched % kSlots);
+    if (!mbar_wait(&s.slot_full[slot], (fetched / kSlots) & 1, &s.abort, kTimeoutNs)) return false;
+    o.flags = s.meta[slot].flags;
+#pragma unroll
+    for (int g = 0; g < G; ++g) o.w[g] = s.meta[slot].w[g];
+    if (!(o.flags & kLastUnit) && (o.flags & use_mask)) {
+      const char* base = reinterpret_cast<const char*>(&s.slot[slot][0]) + row_off;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) o.d[c] = *reinterpret_cast<const uint4*>(base + (((4 * chalf + c) ^ sw) << 4));
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.slot_empty[slot]);
+    ++fetched;
+    return true;
+  };
+
+  unsigned long long acc[G][16];  // pairs of fp32 accumulators: columns (2e, 2e + 1)
+  SlotData cur;
   for (int k = blockIdx.x; k < p.n_units && ok; k += gridDim.x, ++nunit) {
     const Unit u = decode(p, k);
-    bool any = false;
-    // sub-steps until the producer's end-of-unit marker slot
-    bool unit_done = false;
+    bool any = false, unit_done = false;
     while (!unit_done && ok) {
 #pragma unroll
       for (int g = 0; g < G; ++g)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) acc[g][e] = 0.f;
+        for (int e = 0; e < 16; ++e) acc[g][e] = 0ull;
       bool sub_done = false;
       while (!sub_done) {
-        const int slot = (int)(f % kSlots);
-        if (!mbar_wait(&s.slot_full[slot], (f / kSlots) & 1, &s.abort, kTimeoutNs)) {
+        if (!fetch(cur)) {
           fail(s, p, 0x301);
           ok = false;
           break;
         }
-        const uint32_t flags = s.meta[slot].flags;
-        if (flags & kLastUnit) {  // marker slot: no data
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&s.slot_empty[slot]);
-          ++f;
+        const bool marker = (cur.flags & kLastUnit) != 0;
+        if (marker) {
           unit_done = true;
           break;
         }
-        if (flags & (p.B == 128 ? kHalf1 : my_half)) {
-          const char* base = reinterpret_cast<const char*>(&s.slot[slot][0]) + row_off;
-          float w[G];
+        if (cur.flags & use_mask) {
+          unsigned long long w2[G];
 #pragma unroll
-          for (int g = 0; g < G; ++g) w[g] = s.meta[slot].w[g];
+          for (int g = 0; g < G; ++g) w2[g] = pack2(cur.w[g], cur.w[g]);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            const uint4 q = *reinterpret_cast<const uint4*>(base + (((4 * chalf + c) ^ sw) << 4));
-            const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
+            const uint32_t wd[4] = {cur.d[c].x, cur.d[c].y, cur.d[c].z, cur.d[c].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float lo = __uint_as_float(wd[e] << 16);
-              const float hi = __uint_as_float(wd[e] & 0xffff0000u);
+              const unsigned long long v2 =
+                  pack2(__uint_as_float(wd[e] << 16), __uint_as_float(wd[e] & 0xffff0000u));
 #pragma unroll
-              for (int g = 0; g < G; ++g) {
-                acc[g][8 * c + 2 * e] = fmaf(w[g], lo, acc[g][8 * c + 2 * e]);
-                acc[g][8 * c + 2 * e + 1] = fmaf(w[g], hi, acc[g][8 * c + 2 * e + 1]);
-              }
+              for (int g = 0; g < G; ++g) acc[g][4 * c + e] = ffma2(w2[g], v2, acc[g][4 * c + e]);
             }
           }
         }
-        sub_done = (flags & kLastSub) != 0;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.slot_empty[slot]);
-        ++f;
+        sub_done = (cur.flags & kLastSub) != 0;
       }
       if (!ok || unit_done) break;
       any = true;
@@ -482,7 +498,9 @@ __device__ void mixers(Smem& s, const Params& p) {
           uint32_t pk[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[g][8 * c + 2 * e], acc[g][8 * c + 2 * e + 1]);
+            float lo, hi;
+            unpack2(acc[g][4 * c + e], lo, hi);
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);
             pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
           }
           *reinterpret_cast<uint4*>(xb + (((4 * chalf + c) ^ sw) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -562,8 +580,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_retrieve_tc(const __grid_consta
   tc_fence_after();
   if (warp < kMixWarps)
     mixers<G>(s, p);
-  else if (warp == kProducerWarp)
-    producer<G>(s, p, &tmap_v);
+  else if (warp < kProducerWarp0 + kProducers)
+    producer<G>(s, p, &tmap_v, warp - kProducerWarp0);
   else
     mma_issuer<G>(s, p);
   tc_fence_before();
