@@ -30,7 +30,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from cross_model_attention_mr_b200.workloads import config, draw_layers  # noqa: E402
+from cross_model_attention_mr_b200.workloads import config, draw_layers, shrink  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "prefill tokens/s for compress+retrieve at L=32K; % TC peak and % HBM peak"
@@ -240,6 +240,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--L", type=int, default=None,
+                    help="shorter sequence of the same workload shape (profiling captures); default 32768")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -247,6 +249,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     spec = config(4)
+    if args.L is not None and args.L != spec.L:
+        spec = shrink(spec, L=args.L, name=spec.name.replace("L32768", f"L{args.L}"))
 
     if args.impl == "reference":
         run_reference(args, spec, rank)
@@ -324,6 +328,9 @@ def main():
     mr.profile_enable(False)
     launches = mr.kernel_launches() - launches0
     ms = ev0.elapsed_time(ev1) / args.steps
+    st_c, st_r = ws_c.sync_status(), ws_r.sync_status()
+    if st_c or st_r:
+        raise SystemExit(f"device status in the timed steps: compress={st_c} retrieve={st_r}")
     if dist is not None:
         t = torch.tensor([ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)

@@ -460,7 +460,7 @@ __device__ void softmax_group(Smem& s, const Params& p, int w) {
 __global__ void __launch_bounds__(kThreads, 1)
     k_compress_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk, Params p) {
   extern __shared__ unsigned char smem_raw[];
-  Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem& s = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     mbar_init(&s.q_full, 1);

@@ -6,14 +6,18 @@
 // query block of 128, or two consecutive blocks of 64) x G receiver heads x R requests, with
 // G * R = 4 fp32 accumulators of 128 x 128 in Tensor Memory (all 512 columns).  Key blocks are
 // consumed in sub-steps of 64 keys:
-//   * producer warp: for every sender head that kept the key block (bitmask union), bulk-copies
-//     that tile's 64-column panel (a 128-byte-swizzled K-major operand as stored) into a ring of
-//     shared-memory slots, and loads the receivers' V rows with TMA (128-byte swizzle);
-//   * 8 mixer warps: the head mixing as a weighted accumulation in registers (each thread owns
-//     one row and 32 columns for G heads), then write X_r as a bf16 MMA operand to shared memory;
-//     the translated map exists only there, never in global memory;
-//   * MMA warp: tcgen05.mma X_r (128 x 64, K-major) x V (64 x 128, MN-major) into the fp32
-//     accumulators;
+//   * planner warp: for every sender head that kept the key block (bitmask union) writes one
+//     entry (tile index, the unit's mixing weights W[r, s]) into a page of a shared-memory ring,
+//     one page per sub-step, and pulls the sub-step's map panels into L2 ahead of use;
+//   * 16 mixer warps: each thread copies its own 2 x 16 bytes of every listed panel from L2 into
+//     a private shared-memory ring, two panels (sender heads) per slot (cp.async, per-thread
+//     completion: no per-panel barrier), accumulates the head mixing in fp32 (pairs of columns
+//     per FFMA2), and at the end
+//     of a sub-step writes X_r as a bf16 MMA operand to shared memory; the translated map exists
+//     only there, never in global memory;
+//   * MMA warp: loads the receivers' V rows for the next sub-step with TMA (128-byte swizzle)
+//     once the current MMAs have read the buffer, and issues tcgen05.mma X_r (128 x 64, K-major)
+//     x V (64 x 128, MN-major) into the fp32 accumulators;
 //   * epilogue (mixer warps): Tensor Memory -> registers -> bf16 -> global O.
 // Every wait is bounded; a wait that runs out records MR_ERR_TIMEOUT and the CTA drains its
 // in-flight copies and MMAs, frees Tensor Memory and returns.
@@ -30,15 +34,17 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kMixWarps = 8;
-constexpr int kProducerWarp0 = 8;  // producer warps 8, 9, 10 (each owns ring slots p and p + 3)
-constexpr int kProducers = 3;
-constexpr int kMmaWarp = 11;
-constexpr int kThreads = 384;
-constexpr int kSlots = 6;
-constexpr int kSlotBytes = 16384;
+constexpr int kMixWarps = 16;
+constexpr int kPlanWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kThreads = 576;
+constexpr int kMixThreads = kMixWarps * 32;
+constexpr int kQueue = 2;       // entry pairs in flight per mixer thread (its shared-memory ring)
+constexpr int kPages = 12;      // > 2 * kQueue + 2: the fetch cursor never laps the compute cursor
+constexpr int kMaxEntries = 64; // sender heads
 constexpr int kAcc = 4;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr uint32_t kNone = 0xffffffffu;
 
 struct Params {
   const uint32_t* kept_bits;
@@ -54,20 +60,26 @@ struct Params {
   WsHeader* ws;
 };
 
-// What a ring slot holds, written by the producer before the slot's full barrier is armed.
-struct SlotMeta {
-  float w[kAcc];   // W[r][s] of the unit's receiver heads for the slot's sender head s
-  uint32_t flags;  // kHalf0 | kHalf1 | kLastSub | kLastUnit | kEmptyUnit
+// One listed panel: the tile of each of the unit's two query blocks (kNone: not kept, or never
+// stored because the map overflowed) and the unit's mixing weights for the panel's sender head.
+struct Entry {
+  uint32_t t[2];
+  uint32_t pad[2];
+  float w[kAcc];
 };
-constexpr uint32_t kHalf0 = 1u, kHalf1 = 2u, kLastSub = 4u, kLastUnit = 8u, kEmptyUnit = 16u;
+// One sub-step (n >= 1 entries, panel h of the key block) or a marker (n == 0).
+struct Page {
+  uint32_t n, h, flags, pad;
+  Entry e[kMaxEntries];
+};
+constexpr uint32_t kUnitEnd = 1u, kEmptyUnit = 2u, kEnd = 4u;
 
 struct Smem {
-  __nv_bfloat16 slot[kSlots][kSlotBytes / 2];
   __nv_bfloat16 x[kAcc][128 * 64];
   __nv_bfloat16 v[kAcc][64 * 128];
-  SlotMeta meta[kSlots];
-  uint64_t slot_full[kSlots];
-  uint64_t slot_empty[kSlots];
+  uint4 ring[kQueue][2][2][kMixThreads];  // [pair slot][entry of the pair][piece][mixer thread]
+  Page page[kPages];
+  uint64_t plan_full[kPages], plan_empty[kPages];
   uint64_t x_full, x_empty, v_full, v_empty, o_full, o_empty, mma_done;
   uint32_t tmem_base;
   int abort;
@@ -120,7 +132,6 @@ __device__ __forceinline__ void fail(Smem& s, const Params& p, uint32_t detail) 
   s.abort = 1;
 }
 
-// ------------------------------------------------------------------------------------------------
 // Per-lane view of one (sender head, query block) map row while J advances within a unit: the
 // current 32-bit word of kept bits, the number of kept blocks below J, and the row's first tile.
 struct RowCursor {
@@ -151,46 +162,42 @@ struct RowCursor {
   }
 };
 
-// Producer warp `pw` (0..2).  Bulk copies are issued by several warps because one issuing warp
-// is limited to a few million copies per second; each warp fills only the ring slots it owns
-// (slot % 3 == pw), so a slot's fills are always issued by one warp, in order, each after the
-// release of the previous one.  All producer warps walk the same unit / key-block sequence.
+// ------------------------------------------------------------------------------------------------
+// Planner warp: pages (one per sub-step, plus a marker after every unit and one at the end).  It
+// waits only for page slots, never for the tensor core.
 template <int G>
-__device__ void producer(Smem& s, const Params& p, const CUtensorMap* tmap_v, int pw) {
+__device__ void planner(Smem& s, const Params& p) {
   const int lane = threadIdx.x & 31;
-  uint32_t f = 0;   // slot fills in the sequence so far (all warps)
-  uint32_t nv = 0;  // V fills issued (warp 0 only; one per executed sub-step)
-  uint32_t hi = 0;  // one past the last fill this warp issued
+  uint32_t np = 0;    // pages written
   const int nparts = p.B / 64;
   bool ok = true;
 
-  auto issue_v = [&](const Unit& u, int j0) {
-    uint32_t bytes = 0;
-    for (int a = 0; a < G * p.R; ++a)
-      if (acc_valid(p, u, G, a)) bytes += 64 * 128 * 2;
-    mbar_arrive_expect_tx(&s.v_full, bytes);
-    for (int a = 0; a < G * p.R; ++a) {
-      if (!acc_valid(p, u, G, a)) continue;
-      const int r = u.hg * G + a / p.R, q = u.rg * p.R + a % p.R;
-      const int64_t off = (p.v_req_off ? p.v_req_off[q] : (int64_t)q * p.v_req_stride) + (int64_t)r * p.v_head_stride;
-      const int row = (int)(off / 128) + j0;
-      tma_load_2d(&s.v[a][0], tmap_v, &s.v_full, 0, row);
-      tma_load_2d(&s.v[a][64 * 64], tmap_v, &s.v_full, 64, row);
-    }
-    ++nv;
-  };
-  auto owns = [&](uint32_t F) { return (int)((F % kSlots) % kProducers) == pw; };
-  // lane 0 waits until the slot of fill F is free (its previous fill, issued by this warp, released)
-  auto claim = [&](uint32_t F) -> bool {
+  // lane 0 waits until page np's slot was released by every mixer warp
+  auto claim = [&]() -> Page* {
     bool good = true;
-    if (lane == 0 && F >= (uint32_t)kSlots &&
-        !mbar_wait(&s.slot_empty[F % kSlots], ((F / kSlots) - 1) & 1, &s.abort, kTimeoutNs)) {
-      fail(s, p, 0x102);
+    if (lane == 0 && np >= (uint32_t)kPages &&
+        !mbar_wait_sleep(&s.plan_empty[np % kPages], ((np / kPages) - 1) & 1, &s.abort, kTimeoutNs, 256)) {
+      fail(s, p, 0x101);
       good = false;
     }
-    return __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+    ok = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+    return &s.page[np % kPages];
   };
-
+  auto publish = [&]() {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.plan_full[np % kPages]);
+    ++np;
+  };
+  auto marker = [&](uint32_t flags) {
+    Page* pg = claim();
+    if (!ok) return;
+    if (lane == 0) {
+      pg->n = 0;
+      pg->h = 0;
+      pg->flags = flags;
+    }
+    publish();
+  };
   for (int k = blockIdx.x; k < p.n_units && ok; k += gridDim.x) {
     const Unit u = decode(p, k);
     // lane l tracks sender heads l and l + 32, for the unit's one or two query blocks
@@ -220,83 +227,46 @@ __device__ void producer(Smem& s, const Params& p, const CUtensorMap* tmap_v, in
       const uint64_t m0 = ((uint64_t)__ballot_sync(0xffffffffu, b[0][1]) << 32) | __ballot_sync(0xffffffffu, b[0][0]);
       const uint64_t m1 = p.B == 64
                               ? (((uint64_t)__ballot_sync(0xffffffffu, b[1][1]) << 32) | __ballot_sync(0xffffffffu, b[1][0]))
-                              : m0;
+                              : 0ull;
       const uint64_t uni = m0 | m1;
       if (uni != 0) {
-        const int nsl = __popcll((long long)uni);
         for (int h = 0; h < nparts && ok; ++h) {
-          const int j0 = J * p.B + 64 * h;
-          uint64_t rem = uni;
-          for (int rank = 0; rank < nsl && ok; ++rank) {
-            const int sh = __ffsll((long long)rem) - 1;
-            rem &= rem - 1;
-            const uint32_t F = f + (uint32_t)rank;
-            if (!owns(F)) continue;  // warp-uniform
-            if (!claim(F)) {
-              ok = false;
-              break;
-            }
-            const int src_lane = sh & 31, hs = sh >> 5;
-            int64_t t[2];
-            bool use[2];
+          Page* pg = claim();
+          if (!ok) break;
+          // every lane writes the entries of its own sender heads, at their rank in the union
+#pragma unroll
+          for (int hs = 0; hs < 2; ++hs) {
+            const int sh = lane + 32 * hs;
+            if (!((uni >> sh) & 1ull)) continue;
+            const int rank = __popcll((long long)(uni & ((1ull << sh) - 1ull)));
+            Entry& e = pg->e[rank];
 #pragma unroll
             for (int pt = 0; pt < 2; ++pt) {
-              const int64_t t0 = __shfl_sync(0xffffffffu, cur[pt][0].first + cur[pt][0].count, src_lane);
-              const int64_t t1 = __shfl_sync(0xffffffffu, cur[pt][1].first + cur[pt][1].count, src_lane);
-              t[pt] = hs ? t1 : t0;
-              use[pt] = ((pt == 0 ? m0 : m1) >> sh) & 1ull;
-            }
-            float w[kAcc];
-#pragma unroll
-            for (int g = 0; g < kAcc; ++g) {
-              const float w0 = __shfl_sync(0xffffffffu, wv[0][g], src_lane);
-              const float w1 = __shfl_sync(0xffffffffu, wv[1][g], src_lane);
-              w[g] = hs ? w1 : w0;
-            }
-            if (lane == 0) {
-              const int slot = (int)(F % kSlots);
-              char* dst = reinterpret_cast<char*>(&s.slot[slot][0]);
-              uint32_t bytes = 0, flags = 0;
-              const uint32_t len = p.B == 128 ? 16384u : 8192u;
-              const char* src[2] = {nullptr, nullptr};
-              for (int pt = 0; pt < (p.B == 64 ? 2 : 1); ++pt) {
-                if (!use[pt]) continue;
-                flags |= pt == 0 ? kHalf0 : kHalf1;
-                if (t[pt] >= p.capacity) {
-                  // the map overflowed: this tile was never stored; contribute zeros
-                  uint4* z = reinterpret_cast<uint4*>(dst + pt * 8192);
-                  for (uint32_t e = 0; e < len / 16; ++e) z[e] = make_uint4(0, 0, 0, 0);
-                  set_status(p.ws, MR_ERR_CAPACITY, 3u);
+              uint32_t t = kNone;
+              if (b[pt][hs]) {
+                const int64_t tt = cur[pt][hs].first + cur[pt][hs].count;
+                if (tt < p.capacity) {
+                  t = (uint32_t)tt;
+                  const char* src = reinterpret_cast<const char*>(p.vals + tt * (int64_t)p.B * p.B) +
+                                    (p.B == 128 ? 16384 * h : 0);
+                  bulk_prefetch_l2(src, p.B == 128 ? 16384u : 8192u);
                 } else {
-                  src[pt] = reinterpret_cast<const char*>(p.vals + t[pt] * (int64_t)p.B * p.B) + (p.B == 128 ? 16384 * h : 0);
-                  bytes += len;
+                  set_status(p.ws, MR_ERR_CAPACITY, 3u);  // the map overflowed: this tile was never stored
                 }
               }
-              if (p.B == 128) flags |= kHalf1;  // one 128-row panel serves every row
-              if (rank == nsl - 1) flags |= kLastSub;
+              e.t[pt] = t;
+            }
 #pragma unroll
-              for (int g = 0; g < kAcc; ++g) s.meta[slot].w[g] = w[g];
-              s.meta[slot].flags = flags;
-              mbar_arrive_expect_tx(&s.slot_full[slot], bytes);
-              for (int pt = 0; pt < 2; ++pt)
-                if (src[pt]) bulk_g2s(dst + pt * 8192, src[pt], len, &s.slot_full[slot]);
-            }
-            hi = F + 1;
-            __syncwarp();
+            for (int g = 0; g < kAcc; ++g) e.w[g] = wv[hs][g];
           }
-          if (!ok) break;
-          f += (uint32_t)nsl;
-          // V of this sub-step (warp 0), once the previous sub-step's MMAs released the V buffer
-          if (pw == 0 && lane == 0) {
-            if (nv > 0 && !mbar_wait(&s.v_empty, (nv - 1) & 1, &s.abort, kTimeoutNs)) {
-              fail(s, p, 0x101);
-              ok = false;
-            } else {
-              issue_v(u, j0);
-            }
+          if (lane == 0) {
+            const uint32_t n = (uint32_t)__popcll((long long)uni);
+            pg->n = n;
+            pg->h = (uint32_t)h;
+            pg->flags = 0u;
+            if (n & 1u) pg->e[n].t[0] = pg->e[n].t[1] = kNone;  // mixers take entries in pairs
           }
-          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-          nv = __shfl_sync(0xffffffffu, nv, 0);
+          publish();
           any_unit = true;
         }
       }
@@ -307,43 +277,87 @@ __device__ void producer(Smem& s, const Params& p, const CUtensorMap* tmap_v, in
         for (int hs = 0; hs < 2; ++hs) cur[pt][hs].count += b[pt][hs] ? 1 : 0;
     }
     if (!ok) break;
-    // mark the end of the unit with a data-less slot (the unit's only slot if it kept nothing)
-    if (owns(f)) {
-      if (!claim(f)) {
-        ok = false;
-        break;
-      }
-      if (lane == 0) {
-        s.meta[f % kSlots].flags = any_unit ? kLastUnit : (kLastUnit | kEmptyUnit);
-        mbar_arrive(&s.slot_full[f % kSlots]);
-      }
-      hi = f + 1;
-      __syncwarp();
-    }
-    ++f;
+    marker(any_unit ? kUnitEnd : (kUnitEnd | kEmptyUnit));
   }
-  // drain: every copy this warp issued must land before the CTA can release its shared memory
-  if (lane == 0) {
-    const int never = 0;  // drain even after an abort: wait on the copies themselves (bounded)
-    for (uint32_t g = (hi > (uint32_t)kSlots ? hi - kSlots : 0); g < hi; ++g)
-      if (owns(g)) mbar_wait(&s.slot_full[g % kSlots], (g / kSlots) & 1, &never, kTimeoutNs);
-    if (nv > 0) mbar_wait(&s.v_full, (nv - 1) & 1, &never, kTimeoutNs);
-  }
-  __syncwarp();
+  if (ok) marker(kEnd);
 }
 
+// ------------------------------------------------------------------------------------------------
+// Walks the sub-steps (unit, key block J, 64-key panel h) of this CTA in order.  Warp-collective.
+struct SubWalker {
+  int k, J, h;
+  Unit u;
+  bool live;
+  __device__ __forceinline__ void start(const Params& p) {
+    k = blockIdx.x;
+    live = k < p.n_units;
+    if (live) u = decode(p, k);
+    J = 0;
+    h = -1;
+  }
+  // move to the next sub-step; false once the CTA has none left
+  __device__ __forceinline__ bool next(const Params& p) {
+    const int nparts = p.B / 64;
+    while (live) {
+      if (h >= 0 && h + 1 < nparts) {
+        ++h;
+        return true;
+      }
+      if (h >= 0) ++J;
+      h = -1;
+      for (; J <= u.Jmax; ++J) {
+        const uint64_t m0 = head_mask(p, u.I0, J);
+        const uint64_t m1 = (p.B == 64) ? head_mask(p, u.I1, J) : 0ull;
+        if ((m0 | m1) != 0) {
+          h = 0;
+          return true;
+        }
+      }
+      k += gridDim.x;
+      live = k < p.n_units;
+      if (live) u = decode(p, k);
+      J = 0;
+    }
+    return false;
+  }
+};
+
 template <int G>
-__device__ void mma_issuer(Smem& s, const Params& p) {
+__device__ void issue_v(Smem& s, const Params& p, const CUtensorMap* tmap_v, const Unit& u, int j0) {
+  uint32_t bytes = 0;
+  for (int a = 0; a < G * p.R; ++a)
+    if (acc_valid(p, u, G, a)) bytes += 64 * 128 * 2;
+  mbar_arrive_expect_tx(&s.v_full, bytes);
+  for (int a = 0; a < G * p.R; ++a) {
+    if (!acc_valid(p, u, G, a)) continue;
+    const int r = u.hg * G + a / p.R, q = u.rg * p.R + a % p.R;
+    const int64_t off = (p.v_req_off ? p.v_req_off[q] : (int64_t)q * p.v_req_stride) + (int64_t)r * p.v_head_stride;
+    const int row = (int)(off / 128) + j0;
+    tma_load_2d(&s.v[a][0], tmap_v, &s.v_full, 0, row);
+    tma_load_2d(&s.v[a][64 * 64], tmap_v, &s.v_full, 64, row);
+  }
+}
+
+// MMA warp: per sub-step, X (from the mixers) x V (loaded here one sub-step ahead) into the unit's
+// accumulators; the next V load is issued once these MMAs have read the buffer.
+template <int G>
+__device__ void mma_issuer(Smem& s, const Params& p, const CUtensorMap* tmap_v) {
   const int lane = threadIdx.x & 31;
   const uint32_t idesc = idesc_bf16_f32(128, 128, false, true);
   const uint32_t tbase = s.tmem_base;
-  uint32_t nsub = 0;
+  uint32_t nsub = 0, nv = 0;
   int nunit = 0;
   bool ok = true;
   const int nparts = p.B / 64;
+  SubWalker vw;  // the sub-step whose V is loaded next
+  vw.start(p);
+  if (vw.next(p)) {
+    if (lane == 0) issue_v<G>(s, p, tmap_v, vw.u, vw.J * p.B + 64 * vw.h);
+    ++nv;
+  }
   for (int k = blockIdx.x; k < p.n_units && ok; k += gridDim.x, ++nunit) {
     const Unit u = decode(p, k);
-    if (lane == 0 && nunit > 0 && !mbar_wait(&s.o_empty, (nunit - 1) & 1, &s.abort, kTimeoutNs)) {
+    if (lane == 0 && nunit > 0 && !mbar_wait_sleep(&s.o_empty, (nunit - 1) & 1, &s.abort, kTimeoutNs, 64)) {
       fail(s, p, 0x201);
       ok = false;
     }
@@ -352,12 +366,12 @@ __device__ void mma_issuer(Smem& s, const Params& p) {
     bool first = true;
     for (int J = 0; J <= u.Jmax && ok; ++J) {
       const uint64_t m0 = head_mask(p, u.I0, J);
-      const uint64_t m1 = (p.B == 64) ? head_mask(p, u.I1, J) : m0;
+      const uint64_t m1 = (p.B == 64) ? head_mask(p, u.I1, J) : 0ull;
       if ((m0 | m1) == 0) continue;
       for (int h = 0; h < nparts && ok; ++h) {
         if (lane == 0) {
-          if (!mbar_wait(&s.x_full, nsub & 1, &s.abort, kTimeoutNs) ||
-              !mbar_wait(&s.v_full, nsub & 1, &s.abort, kTimeoutNs)) {
+          if (!mbar_wait_sleep(&s.x_full, nsub & 1, &s.abort, kTimeoutNs, 64) ||
+              !mbar_wait_sleep(&s.v_full, nsub & 1, &s.abort, kTimeoutNs, 64)) {
             fail(s, p, 0x202);
             ok = false;
           } else {
@@ -381,6 +395,20 @@ __device__ void mma_issuer(Smem& s, const Params& p) {
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         first = false;
         ++nsub;
+        if (!ok) break;
+        // the next sub-step's V, once these MMAs have read the buffer
+        if (vw.next(p)) {
+          if (lane == 0) {
+            if (!mbar_wait_sleep(&s.v_empty, (nsub - 1) & 1, &s.abort, kTimeoutNs, 64)) {
+              fail(s, p, 0x203);
+              ok = false;
+            } else {
+              issue_v<G>(s, p, tmap_v, vw.u, vw.J * p.B + 64 * vw.h);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (ok) ++nv;
+        }
       }
     }
     if (ok && lane == 0) {
@@ -391,147 +419,188 @@ __device__ void mma_issuer(Smem& s, const Params& p) {
     }
     __syncwarp();
   }
-  // drain: all MMAs issued by this thread complete before Tensor Memory is released
+  // drain: all MMAs issued by this thread complete before Tensor Memory is released, and the
+  // last V load lands before shared memory is
   if (lane == 0) {
     mma_commit(&s.mma_done);
     const int never = 0;
     mbar_wait(&s.mma_done, 0, &never, kTimeoutNs);
+    if (nv > 0) mbar_wait(&s.v_full, (nv - 1) & 1, &never, kTimeoutNs);
   }
   __syncwarp();
 }
 
 // ------------------------------------------------------------------------------------------------
-// What a mixer thread takes from one ring slot: the slot's flags and weights and its own 32
-// columns of its own row (4 x 16 bytes).
-struct SlotData {
-  uint32_t flags;
-  float w[kAcc];
-  uint4 d[4];
-};
+// 16-byte global -> shared copy through L2 only, completed per thread by cp.async.wait_group
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
+  return v;
+}
 
+// Mixer warp w owns unit rows 8w .. 8w + 7.  Thread (w, l) owns rows a_k = 8w + 4k + l/8 (k = 0, 1)
+// and, in each, the 16-byte chunk at physical position l % 8 of the 128-byte-swizzled panel row:
+// eight consecutive keys 8 * ((l % 8) ^ (a_k % 8)).  X is written with the same swizzle, so the
+// thread writes its chunks back to the positions it read them from.
 template <int G>
 __device__ void mixers(Smem& s, const Params& p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = 32 * (warp & 3) + lane;  // 0..127: this thread's query row within the unit
-  const int chalf = warp >> 2;             // which 32 of the sub-step's 64 columns
-  const int half = row >> 6;               // for 64-key blocks: which of the two query blocks
-  const uint32_t use_mask = (p.B == 128) ? kHalf1 : (half ? kHalf1 : kHalf0);
-  const uint32_t row_off = (p.B == 64) ? (uint32_t)(half * 8192 + (row & 63) * 128) : (uint32_t)(row * 128);
-  const int sw = row & 7;
+  const int half = p.B == 64 ? (warp >> 3) : 0;  // 64-key blocks: which of the unit's two query blocks
+  const uint32_t rowb = (uint32_t)(8 * warp + (lane >> 3));
+  const uint32_t my_off = (p.B == 64 ? (rowb & 63u) : rowb) * 128u + (uint32_t)(lane & 7) * 16u;  // bytes
+  const uint32_t tile_bytes = (uint32_t)(p.B * p.B * 2);
+  const char* vals = reinterpret_cast<const char*>(p.vals);
   const uint32_t tbase = s.tmem_base;
-  uint32_t fetched = 0, nsub = 0;
-  int nunit = 0;
-  bool ok = true;
+  const int tw = warp & 3;  // Tensor Memory lane quadrant of this warp
 
-  // Wait for the next fill, copy what this thread needs into registers, and hand the slot back
-  // to the producer at once (the arrive orders the reads before any refill).
-  auto fetch = [&](SlotData& o) -> bool {
-    const int slot = (int)(fetched % kSlots);
-    if (!mbar_wait(&s.slot_full[slot], (fetched / kSlots) & 1, &s.abort, kTimeoutNs)) return false;
-    o.flags = s.meta[slot].flags;
-#pragma unroll
-    for (int g = 0; g < G; ++g) o.w[g] = s.meta[slot].w[g];
-    if (!(o.flags & kLastUnit) && (o.flags & use_mask)) {
-      const char* base = reinterpret_cast<const char*>(&s.slot[slot][0]) + row_off;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) o.d[c] = *reinterpret_cast<const uint4*>(base + (((4 * chalf + c) ^ sw) << 4));
-    }
+  // Fetch cursor (kQueue entry pairs ahead) and compute cursor over the page ring; a page of n
+  // entries is taken as (n + 1) / 2 pairs (the planner pads odd pages with an empty entry).
+  uint32_t pf = 0, ef = 0, nf = 0, hf = 0;  // page, pair, pairs in page, panel
+  bool f_done = false;
+  uint32_t pc = 0, ec = 0, nc = 0;
+  const Page* cpg = &s.page[0];
+  const Page* fpg = &s.page[0];
+  uint32_t nsub = 0;
+  int nunit = 0;
+
+  auto wait_page = [&](uint32_t pg) -> bool {
+    return mbar_wait(&s.plan_full[pg % kPages], (pg / kPages) & 1, &s.abort, kTimeoutNs);
+  };
+  auto release_page = [&](uint32_t pg) {
     __syncwarp();
-    if (lane == 0) mbar_arrive(&s.slot_empty[slot]);
-    ++fetched;
-    return true;
+    if (lane == 0) mbar_arrive(&s.plan_empty[pg % kPages]);
+  };
+  // move the fetch cursor to the next page that lists panels (skipping markers); false on timeout
+  auto fetch_seek = [&](uint32_t from) -> bool {
+    for (uint32_t pg = from;; ++pg) {
+      if (!wait_page(pg)) return false;
+      const Page* P = &s.page[pg % kPages];
+      const uint32_t n = P->n;
+      if (n > 0) {
+        pf = pg;
+        fpg = P;
+        ef = 0;
+        nf = (n + 1) >> 1;
+        hf = P->h;
+        return true;
+      }
+      if (P->flags & kEnd) {
+        f_done = true;
+        return true;
+      }
+    }
+  };
+  // copy the next pair's pieces into ring slot `slot` (one cp.async group per pair, empty when
+  // there is nothing to copy, so group counts stay aligned with pairs); the move to the
+  // following page is taken lazily, at the next call
+  const uint32_t ring0 = smem_u32(&s.ring[0][0][0][threadIdx.x]);
+  constexpr uint32_t kPiece = kMixThreads * 16u, kEntry = 2u * kPiece, kSlot = 2u * kEntry;
+  auto fetch = [&](uint32_t slot) -> bool {
+    bool good = true;
+    if (!f_done && ef == nf) good = fetch_seek(pf + 1);
+    if (good && !f_done) {
+      const uint32_t t0 = fpg->e[2 * ef].t[half], t1 = fpg->e[2 * ef + 1].t[half];
+      const uint32_t dst = ring0 + slot * kSlot;
+      const uint32_t panel = hf * 16384u + my_off;
+      if (t0 != kNone) {
+        const char* src = vals + ((uint64_t)t0 * tile_bytes + panel);
+        cp_async16(dst, src);
+        cp_async16(dst + kPiece, src + 512);
+      }
+      if (t1 != kNone) {
+        const char* src = vals + ((uint64_t)t1 * tile_bytes + panel);
+        cp_async16(dst + kEntry, src);
+        cp_async16(dst + kEntry + kPiece, src + 512);
+      }
+      ++ef;
+    }
+    cp_async_commit();
+    return good;
   };
 
-  unsigned long long acc[G][16];  // pairs of fp32 accumulators: columns (2e, 2e + 1)
-  SlotData cur;
-  for (int k = blockIdx.x; k < p.n_units && ok; k += gridDim.x, ++nunit) {
-    const Unit u = decode(p, k);
-    bool any = false, unit_done = false;
-    while (!unit_done && ok) {
+  unsigned long long acc[G][8];  // pairs of fp32 accumulators: columns (2e, 2e + 1) of the thread's chunks
 #pragma unroll
-      for (int g = 0; g < G; ++g)
+  for (int g = 0; g < G; ++g)
 #pragma unroll
-        for (int e = 0; e < 16; ++e) acc[g][e] = 0ull;
-      bool sub_done = false;
-      while (!sub_done) {
-        if (!fetch(cur)) {
-          fail(s, p, 0x301);
-          ok = false;
-          break;
-        }
-        const bool marker = (cur.flags & kLastUnit) != 0;
-        if (marker) {
-          unit_done = true;
-          break;
-        }
-        if (cur.flags & use_mask) {
-          unsigned long long w2[G];
+    for (int e = 0; e < 8; ++e) acc[g][e] = 0ull;
+
+  // one entry: acc[g] += W[r_g, s] * (this thread's 16 values of the sender head's panel)
+  auto mix_entry = [&](const Entry& E, uint32_t data) {
+    const float4 wf = *reinterpret_cast<const float4*>(&E.w[0]);
+    const float w[4] = {wf.x, wf.y, wf.z, wf.w};
+    unsigned long long w2[G];
 #pragma unroll
-          for (int g = 0; g < G; ++g) w2[g] = pack2(cur.w[g], cur.w[g]);
+    for (int g = 0; g < G; ++g) w2[g] = pack2(w[g], w[g]);
+    const uint4 d0 = lds128(data), d1 = lds128(data + kPiece);
+    const uint32_t wd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+    if constexpr (G == 4) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint32_t wd[4] = {cur.d[c].x, cur.d[c].y, cur.d[c].z, cur.d[c].w};
+      for (int e = 0; e < 8; ++e)
+        mix_word4(acc[0][e], acc[1][e], acc[2][e], acc[3][e], wd[e], w2[0], w2[1], w2[2], w2[3]);
+    } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const unsigned long long v2 =
-                  pack2(__uint_as_float(wd[e] << 16), __uint_as_float(wd[e] & 0xffff0000u));
+      for (int e = 0; e < 8; ++e) {
+        const unsigned long long v2 = pack2(__uint_as_float(wd[e] << 16), __uint_as_float(wd[e] & 0xffff0000u));
 #pragma unroll
-              for (int g = 0; g < G; ++g) acc[g][4 * c + e] = ffma2(w2[g], v2, acc[g][4 * c + e]);
-            }
-          }
-        }
-        sub_done = (cur.flags & kLastSub) != 0;
+        for (int g = 0; g < G; ++g) acc[g][e] = ffma2(w2[g], v2, acc[g][e]);
       }
-      if (!ok || unit_done) break;
-      any = true;
-      // hand X to the tensor core once the previous sub-step's MMAs have read it
-      if (nsub > 0 && !mbar_wait(&s.x_empty, (nsub - 1) & 1, &s.abort, kTimeoutNs)) {
-        fail(s, p, 0x302);
-        ok = false;
-        break;
-      }
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        char* xb = reinterpret_cast<char*>(&s.x[g][0]) + row * 128;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float lo, hi;
-            unpack2(acc[g][4 * c + e], lo, hi);
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);
-            pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
-          }
-          *reinterpret_cast<uint4*>(xb + (((4 * chalf + c) ^ sw) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.x_full);
-      ++nsub;
     }
-    if (!ok) break;
-    // ---- epilogue: accumulators -> bf16 -> O ----
-    if (!mbar_wait(&s.o_full, nunit & 1, &s.abort, kTimeoutNs)) {
-      fail(s, p, 0x303);
-      ok = false;
-      break;
+  };
+
+  // X of one sub-step, once the previous sub-step's MMAs have read the buffer
+  auto hand_x = [&]() -> bool {
+    if (nsub > 0 && !mbar_wait(&s.x_empty, (nsub - 1) & 1, &s.abort, kTimeoutNs)) return false;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float lo, hi;
+          unpack2(acc[g][4 * k + e], lo, hi);
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);
+          pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
+          acc[g][4 * k + e] = 0ull;
+        }
+        char* xb = reinterpret_cast<char*>(&s.x[g][0]) + (rowb + 4 * k) * 128 + (lane & 7) * 16;
+        *reinterpret_cast<uint4*>(xb) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
     }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.x_full);
+    ++nsub;
+    return true;
+  };
+  // the unit's accumulators -> bf16 -> O (warp w stores accumulator w / 4 of its 32 rows)
+  auto epilogue = [&](bool any) -> bool {
+    if (!mbar_wait(&s.o_full, nunit & 1, &s.abort, kTimeoutNs)) return false;
     tc_fence_after();
+    const Unit u = decode(p, blockIdx.x + nunit * gridDim.x);
+    const int a = warp >> 2;
+    const int row = 32 * tw + lane;
     const int i = u.rb * 128 + row;
-    for (int a = chalf; a < G * p.R; a += 2) {
+    if (a < G * p.R) {
       const bool valid = acc_valid(p, u, G, a);
       const int r = u.hg * G + a / p.R, q = u.rg * p.R + a % p.R;
       __nv_bfloat16* orow = p.O + (((size_t)q * p.H_r + r) * p.L + i) * 128;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(tbase + ((uint32_t)(32 * (warp & 3)) << 16) + 128 * a + 32 * cc, v);
+#pragma unroll 1
+      for (int cc = 0; cc < 8; ++cc) {
+        uint32_t v[16];
+        tmem_ld16(tbase + ((uint32_t)(32 * tw) << 16) + 128 * a + 16 * cc, v);
         tmem_wait_ld();
         if (valid && i < p.L) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < 2; ++c) {
             uint32_t pk[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -540,7 +609,7 @@ __device__ void mixers(Smem& s, const Params& p) {
               const __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
               pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
             }
-            *reinterpret_cast<uint4*>(orow + 32 * cc + 8 * c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(orow + 16 * cc + 8 * c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         }
       }
@@ -548,18 +617,76 @@ __device__ void mixers(Smem& s, const Params& p) {
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.o_empty);
+    ++nunit;
+    return true;
+  };
+  // process marker pages from pc on until a page that lists panels (or the end); false = stop
+  auto compute_seek = [&](bool& stop) -> bool {
+    for (;;) {
+      if (!wait_page(pc)) return false;
+      const Page* P = &s.page[pc % kPages];
+      const uint32_t n = P->n, fl = P->flags;
+      if (n > 0) {
+        cpg = P;
+        ec = 0;
+        nc = (n + 1) >> 1;
+        return true;
+      }
+      if (fl & kUnitEnd) {
+        if (!epilogue(!(fl & kEmptyUnit))) return false;
+      }
+      if (fl & kEnd) {
+        stop = true;
+        return true;
+      }
+      release_page(pc);
+      ++pc;
+    }
+  };
+
+  bool stop = false;
+  bool good = fetch_seek(0) && compute_seek(stop);
+  for (uint32_t u = 0; u < (uint32_t)kQueue; ++u)
+    if (good && !stop) good = fetch(u);
+  uint32_t slot = 0;
+  while (good && !stop) {
+    cp_async_wait<kQueue - 1>();  // this thread's copies of the oldest pair have landed
+    const uint32_t data = ring0 + slot * kSlot;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const Entry& E = cpg->e[2 * ec + j];
+      if (E.t[half] != kNone) mix_entry(E, data + j * kEntry);
+    }
+    if (++ec == nc) {
+      // end of the sub-step: hand X to the tensor core, release the page, run any markers
+      if (!hand_x()) {
+        good = false;
+        break;
+      }
+      release_page(pc);
+      ++pc;
+      if (!compute_seek(stop)) {
+        good = false;
+        break;
+      }
+    }
+    // refill this slot kQueue pairs ahead
+    if (!stop) good = fetch(slot);
+    slot = (slot + 1 == (uint32_t)kQueue) ? 0u : slot + 1;
   }
+  cp_async_wait<0>();  // no copy may land after the CTA releases its shared memory
+  if (!good) fail(s, p, 0x301);
 }
 
 template <int G>
 __global__ void __launch_bounds__(kThreads, 1) k_retrieve_tc(const __grid_constant__ CUtensorMap tmap_v, Params p) {
   extern __shared__ unsigned char smem_raw[];
-  Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem& s = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kSlots; ++i) {
-      mbar_init(&s.slot_full[i], 1);
-      mbar_init(&s.slot_empty[i], kMixWarps);
+    for (int i = 0; i < kPages; ++i) {
+      mbar_init(&s.plan_full[i], 1);
+      mbar_init(&s.plan_empty[i], kMixWarps);
     }
     mbar_init(&s.x_full, kMixWarps);
     mbar_init(&s.x_empty, 1);
@@ -580,10 +707,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_retrieve_tc(const __grid_consta
   tc_fence_after();
   if (warp < kMixWarps)
     mixers<G>(s, p);
-  else if (warp < kProducerWarp0 + kProducers)
-    producer<G>(s, p, &tmap_v, warp - kProducerWarp0);
+  else if (warp == kPlanWarp)
+    planner<G>(s, p);
   else
-    mma_issuer<G>(s, p);
+    mma_issuer<G>(s, p, &tmap_v);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -604,7 +731,8 @@ cudaError_t launch_g(const RetrieveArgs& a, const Params& p, const CUtensorMap& 
 
 bool tc_retrieve_supported(const RetrieveArgs& a) {
   return a.dt == MR_BF16 && a.d_v == 128 && (a.map.block == 64 || a.map.block == 128) && a.map.H_s <= 64 &&
-         a.v_head_stride % 128 == 0 && (a.v_req_off != nullptr || a.v_req_stride % 128 == 0);
+         a.map.capacity_tiles < (int64_t)kNone && a.v_head_stride % 128 == 0 &&
+         (a.v_req_off != nullptr || a.v_req_stride % 128 == 0);
 }
 
 cudaError_t tc_retrieve(const RetrieveArgs& a) {

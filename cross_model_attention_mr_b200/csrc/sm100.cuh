@@ -65,6 +65,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// As mbar_wait, for warps that mostly wait (producers, MMA issuers): sleeps between polls so the
+// warps that share its SM sub-partition keep the issue slots.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, const volatile int* abort,
+                                                uint64_t timeout_ns, uint32_t sleep_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(sleep_ns);
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+  }
+}
+
 // ------------------------------------------------------------------------------------------------
 // Async proxy copies (no cluster multicast anywhere)
 // ------------------------------------------------------------------------------------------------
@@ -141,6 +155,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t& r) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
 }
@@ -171,6 +194,19 @@ __device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsign
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
+// acc[g] += w2[g] * (lo, hi) for the two bf16 values packed in `x` (low half = lower column),
+// g = 0..3: one word unpacked once, pairs formed in registers (no moves), four FFMA2.
+__device__ __forceinline__ void mix_word4(unsigned long long& a0, unsigned long long& a1, unsigned long long& a2,
+                                          unsigned long long& a3, uint32_t x, unsigned long long w0,
+                                          unsigned long long w1, unsigned long long w2, unsigned long long w3) {
+  asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 v;\n\t"
+      "shl.b32 lo, %4, 16;\n\tand.b32 hi, %4, 0xffff0000;\n\tmov.b64 v, {lo, hi};\n\t"
+      "fma.rn.f32x2 %0, %5, v, %0;\n\tfma.rn.f32x2 %1, %6, v, %1;\n\t"
+      "fma.rn.f32x2 %2, %7, v, %2;\n\tfma.rn.f32x2 %3, %8, v, %3;\n\t}"
+      : "+l"(a0), "+l"(a1), "+l"(a2), "+l"(a3)
+      : "r"(x), "l"(w0), "l"(w1), "l"(w2), "l"(w3));
+}
+
 __device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
   unsigned long long d;
   asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));

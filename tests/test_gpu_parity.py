@@ -30,9 +30,18 @@ def run_layer(mr, spec, lay, capacity=None, p=None):
     st = m.ws.sync_status()
     W = torch.from_numpy(lay.W).cuda()
     V = dev(lay.V, spec.dtype)
-    O = mr.retrieve(m, W, V)
+    ws_r = mr.Workspace(mr.retrieve_workspace_bytes(m, spec.H_r, spec.d_v, 1))
+    O = mr.retrieve(m, W, V, ws=ws_r)
     torch.cuda.synchronize()
+    check_retrieve_status(mr, ws_r, st)
     return m, O, st
+
+
+def check_retrieve_status(mr, ws_r, st_compress=0):
+    """The retrieval's own status word: OK, or CAPACITY when the map it reads overflowed."""
+    st = ws_r.sync_status()
+    allowed = (mr.MR_OK, mr.MR_ERR_CAPACITY) if st_compress == mr.MR_ERR_CAPACITY else (mr.MR_OK,)
+    assert st in allowed, mr.LIB.mr_status_string(st)
 
 
 CASES = {
@@ -96,6 +105,17 @@ def test_single_sender_head_identity_map(mr):
     assert err <= OUT_TOL["bf16"] * float(np.abs(lay.V).max())
 
 
+@pytest.mark.parametrize("n,H_s,H_r", [(2, 1, 1), (2, 1, 5), (4, 1, 4), (4, 2, 3)])
+def test_one_or_two_sender_heads_long_units(mr, n, H_s, H_r):
+    """One or two kept heads per key block: sub-steps of one or two panels, many per unit, so the
+    retrieval's page ring, register queue and double-buffered V run far ahead of the MMAs."""
+    spec = shrink(config(n), L=1536, H_s=H_s, H_r=H_r)
+    lay = draw_layers(spec)[0]
+    m, O, st = run_layer(mr, spec, lay)
+    assert st == mr.MR_OK
+    compare_retrieve(spec, lay, m, O, np.arange(0, spec.L, 7))
+
+
 def test_capacity_overflow_is_reported(mr):
     spec = shrink(config(2), L=512, H_s=2, H_r=2)
     lay = draw_layers(spec)[0]
@@ -125,9 +145,11 @@ def test_multi_request_and_packed_values(mr):
     m = mr.compress(Qs, Ks, p32(spec.p), spec.block, bias=mr.Bias.from_spec(b.bias), scale=spec.scale)
     Vd = dev(Vp, "bf16")
     off = torch.tensor(cu[:-1] * spec.d_v, dtype=torch.int64, device="cuda")
+    ws_r = mr.Workspace(mr.retrieve_workspace_bytes(m, spec.H_r, spec.d_v, 3))
     O = mr.retrieve(m, torch.from_numpy(b.W).cuda(), Vd, v_req_off=off, v_head_stride=int(cu[-1]) * spec.d_v,
-                    n_req=3)
+                    n_req=3, ws=ws_r)
     torch.cuda.synchronize()
+    check_retrieve_status(mr, ws_r)
     rows = np.array([0, 1, 63, 64, 300, 511])
     for q in range(3):
         lay = Layer(Q=b.Qs, K=b.Ks, V=np.ascontiguousarray(b.requests[q].V[:, :P]), W=b.W, bias=b.bias)
