@@ -9,7 +9,7 @@
 //   * planner warp: for every sender head that kept the key block (bitmask union) writes one
 //     entry (tile index, the unit's mixing weights W[r, s]) into a page of a shared-memory ring,
 //     one page per sub-step, and pulls the sub-step's map panels into L2 ahead of use;
-//   * 16 mixer warps: each thread copies its own 2 x 16 bytes of every listed panel from L2 into
+//   * 8 mixer warps: each thread copies its own 4 x 16 bytes of every listed panel from L2 into
 //     a private shared-memory ring, two panels (sender heads) per slot (cp.async, per-thread
 //     completion: no per-panel barrier), accumulates the head mixing in fp32 (pairs of columns
 //     per FFMA2), and at the end
@@ -34,11 +34,15 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kMixWarps = 16;
-constexpr int kPlanWarp = 16;
-constexpr int kMmaWarp = 17;
-constexpr int kThreads = 576;
+// 8 mixer warps + planner + MMA warp: at most 3 warps share an SM sub-partition, so a thread may
+// hold 168 registers, room for 4 x 32 fp32 accumulators without spilling.
+constexpr int kMixWarps = 8;
+constexpr int kPlanWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
 constexpr int kMixThreads = kMixWarps * 32;
+constexpr int kRowsW = 128 / kMixWarps;                  // unit rows per mixer warp
+constexpr int kPieces = 128 * 8 / kMixThreads;           // 16-byte pieces per thread per panel
 constexpr int kQueue = 2;       // entry pairs in flight per mixer thread (its shared-memory ring)
 constexpr int kPages = 12;      // > 2 * kQueue + 2: the fetch cursor never laps the compute cursor
 constexpr int kMaxEntries = 64; // sender heads
@@ -77,7 +81,7 @@ constexpr uint32_t kUnitEnd = 1u, kEmptyUnit = 2u, kEnd = 4u;
 struct Smem {
   __nv_bfloat16 x[kAcc][128 * 64];
   __nv_bfloat16 v[kAcc][64 * 128];
-  uint4 ring[kQueue][2][2][kMixThreads];  // [pair slot][entry of the pair][piece][mixer thread]
+  uint4 ring[kQueue][2][kPieces][kMixThreads];  // [pair slot][entry of the pair][piece][mixer thread]
   Page page[kPages];
   uint64_t plan_full[kPages], plan_empty[kPages];
   uint64_t x_full, x_empty, v_full, v_empty, o_full, o_empty, mma_done;
@@ -446,15 +450,15 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return v;
 }
 
-// Mixer warp w owns unit rows 8w .. 8w + 7.  Thread (w, l) owns rows a_k = 8w + 4k + l/8 (k = 0, 1)
-// and, in each, the 16-byte chunk at physical position l % 8 of the 128-byte-swizzled panel row:
-// eight consecutive keys 8 * ((l % 8) ^ (a_k % 8)).  X is written with the same swizzle, so the
-// thread writes its chunks back to the positions it read them from.
+// Mixer warp w owns unit rows 16w .. 16w + 15.  Thread (w, l) owns rows a_k = 16w + 4k + l/8
+// (k = 0..3) and, in each, the 16-byte chunk at physical position l % 8 of the 128-byte-swizzled
+// panel row: eight consecutive keys 8 * ((l % 8) ^ (a_k % 8)).  X is written with the same
+// swizzle, so the thread writes its chunks back to the positions it read them from.
 template <int G>
 __device__ void mixers(Smem& s, const Params& p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int half = p.B == 64 ? (warp >> 3) : 0;  // 64-key blocks: which of the unit's two query blocks
-  const uint32_t rowb = (uint32_t)(8 * warp + (lane >> 3));
+  const int half = p.B == 64 ? (warp / (kMixWarps / 2)) : 0;  // 64-key blocks: which of the unit's two query blocks
+  const uint32_t rowb = (uint32_t)(kRowsW * warp + (lane >> 3));
   const uint32_t my_off = (p.B == 64 ? (rowb & 63u) : rowb) * 128u + (uint32_t)(lane & 7) * 16u;  // bytes
   const uint32_t tile_bytes = (uint32_t)(p.B * p.B * 2);
   const char* vals = reinterpret_cast<const char*>(p.vals);
@@ -502,7 +506,7 @@ __device__ void mixers(Smem& s, const Params& p) {
   // there is nothing to copy, so group counts stay aligned with pairs); the move to the
   // following page is taken lazily, at the next call
   const uint32_t ring0 = smem_u32(&s.ring[0][0][0][threadIdx.x]);
-  constexpr uint32_t kPiece = kMixThreads * 16u, kEntry = 2u * kPiece, kSlot = 2u * kEntry;
+  constexpr uint32_t kPiece = kMixThreads * 16u, kEntry = kPieces * kPiece, kSlot = 2u * kEntry;
   auto fetch = [&](uint32_t slot) -> bool {
     bool good = true;
     if (!f_done && ef == nf) good = fetch_seek(pf + 1);
@@ -512,13 +516,13 @@ __device__ void mixers(Smem& s, const Params& p) {
       const uint32_t panel = hf * 16384u + my_off;
       if (t0 != kNone) {
         const char* src = vals + ((uint64_t)t0 * tile_bytes + panel);
-        cp_async16(dst, src);
-        cp_async16(dst + kPiece, src + 512);
+#pragma unroll
+        for (int k = 0; k < kPieces; ++k) cp_async16(dst + k * kPiece, src + 512 * k);
       }
       if (t1 != kNone) {
         const char* src = vals + ((uint64_t)t1 * tile_bytes + panel);
-        cp_async16(dst + kEntry, src);
-        cp_async16(dst + kEntry + kPiece, src + 512);
+#pragma unroll
+        for (int k = 0; k < kPieces; ++k) cp_async16(dst + kEntry + k * kPiece, src + 512 * k);
       }
       ++ef;
     }
@@ -526,11 +530,12 @@ __device__ void mixers(Smem& s, const Params& p) {
     return good;
   };
 
-  unsigned long long acc[G][8];  // pairs of fp32 accumulators: columns (2e, 2e + 1) of the thread's chunks
+  constexpr int kW = 4 * kPieces;  // packed bf16 pairs per thread per panel
+  unsigned long long acc[G][kW];   // pairs of fp32 accumulators: columns (2e, 2e + 1) of the thread's chunks
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[g][e] = 0ull;
+    for (int e = 0; e < kW; ++e) acc[g][e] = 0ull;
 
   // one entry: acc[g] += W[r_g, s] * (this thread's 16 values of the sender head's panel)
   auto mix_entry = [&](const Entry& E, uint32_t data) {
@@ -539,18 +544,20 @@ __device__ void mixers(Smem& s, const Params& p) {
     unsigned long long w2[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) w2[g] = pack2(w[g], w[g]);
-    const uint4 d0 = lds128(data), d1 = lds128(data + kPiece);
-    const uint32_t wd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-    if constexpr (G == 4) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
-        mix_word4(acc[0][e], acc[1][e], acc[2][e], acc[3][e], wd[e], w2[0], w2[1], w2[2], w2[3]);
-    } else {
+    for (int k = 0; k < kPieces; ++k) {
+      const uint4 d = lds128(data + k * kPiece);
+      const uint32_t wd[4] = {d.x, d.y, d.z, d.w};
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const unsigned long long v2 = pack2(__uint_as_float(wd[e] << 16), __uint_as_float(wd[e] & 0xffff0000u));
+      for (int e = 0; e < 4; ++e) {
+        const int c = 4 * k + e;
+        if constexpr (G == 4) {
+          mix_word4(acc[0][c], acc[1][c], acc[2][c], acc[3][c], wd[e], w2[0], w2[1], w2[2], w2[3]);
+        } else {
+          const unsigned long long v2 = pack2(__uint_as_float(wd[e] << 16), __uint_as_float(wd[e] & 0xffff0000u));
 #pragma unroll
-        for (int g = 0; g < G; ++g) acc[g][e] = ffma2(w2[g], v2, acc[g][e]);
+          for (int g = 0; g < G; ++g) acc[g][c] = ffma2(w2[g], v2, acc[g][c]);
+        }
       }
     }
   };
@@ -561,7 +568,7 @@ __device__ void mixers(Smem& s, const Params& p) {
 #pragma unroll
     for (int g = 0; g < G; ++g) {
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
+      for (int k = 0; k < kPieces; ++k) {
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -581,15 +588,15 @@ __device__ void mixers(Smem& s, const Params& p) {
     ++nsub;
     return true;
   };
-  // the unit's accumulators -> bf16 -> O (warp w stores accumulator w / 4 of its 32 rows)
+  // the unit's accumulators -> bf16 -> O (warp w stores accumulators w / 4 + 2 i of its 32 rows)
   auto epilogue = [&](bool any) -> bool {
     if (!mbar_wait(&s.o_full, nunit & 1, &s.abort, kTimeoutNs)) return false;
     tc_fence_after();
     const Unit u = decode(p, blockIdx.x + nunit * gridDim.x);
-    const int a = warp >> 2;
     const int row = 32 * tw + lane;
     const int i = u.rb * 128 + row;
-    if (a < G * p.R) {
+#pragma unroll 1
+    for (int a = warp >> 2; a < G * p.R; a += kMixWarps / 4) {
       const bool valid = acc_valid(p, u, G, a);
       const int r = u.hg * G + a / p.R, q = u.rg * p.R + a % p.R;
       __nv_bfloat16* orow = p.O + (((size_t)q * p.H_r + r) * p.L + i) * 128;
