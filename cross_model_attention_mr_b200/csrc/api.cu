@@ -141,7 +141,7 @@ size_t mr_retrieve_workspace_bytes(const mr_bsr* map, int H_r, int d_v, int n_re
   (void)H_r;
   (void)d_v;
   (void)n_req;
-  return kWsHeaderBytes;
+  return kRetrieveWsBytes;
 }
 
 mr_status mr_retrieve(const mr_bsr* map, const float* W, int H_r, const void* V, void* O,
@@ -159,7 +159,7 @@ mr_status mr_retrieve(const mr_bsr* map, const float* W, int H_r, const void* V,
   if (v_head_stride < (int64_t)map->L * d_v) return MR_ERR_INVALID_ARG;
   if (ws_bytes < mr_retrieve_workspace_bytes(map, H_r, d_v, n_req)) return MR_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
-  if (reset_header(ws, st) != cudaSuccess) return MR_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, kRetrieveWsBytes, st) != cudaSuccess) return MR_ERR_CUDA;  // header + progress
   RetrieveArgs a;
   a.map = *map;
   a.W = W;

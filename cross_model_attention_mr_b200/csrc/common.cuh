@@ -17,6 +17,10 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == 64, "header layout");
 constexpr size_t kWsHeaderBytes = 256;
+// Retrieval workspace after the header: one progress counter per CTA (pages consumed), read by
+// the other CTAs of its schedule group to keep the group together.
+constexpr int kMaxProgressCtas = 1024;
+constexpr size_t kRetrieveWsBytes = kWsHeaderBytes + kMaxProgressCtas * sizeof(uint32_t);
 
 __device__ __forceinline__ void set_status(WsHeader* ws, uint32_t code, uint32_t detail) {
   if (atomicCAS(&ws->status, 0u, code) == 0u) ws->detail = detail;

@@ -46,6 +46,8 @@ constexpr int kPieces = 128 * 8 / kMixThreads;           // 16-byte pieces per t
 constexpr int kQueue = 2;       // entry pairs in flight per mixer thread (its shared-memory ring)
 constexpr int kPages = 12;      // > 2 * kQueue + 2: the fetch cursor never laps the compute cursor
 constexpr int kMaxEntries = 64; // sender heads
+constexpr int kPaceSlack = 4;   // pages a CTA may run ahead of the slowest CTA of its group
+constexpr uint64_t kPaceNs = 100000ull;  // longest hold per page
 constexpr int kAcc = 4;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr uint32_t kNone = 0xffffffffu;
@@ -61,6 +63,9 @@ struct Params {
   int64_t v_req_stride, v_head_stride;
   int H_s, H_r, L, B, nqb, nkw, n_req;
   int R, n_hg, n_rg, n_rb, n_units;
+  int per;      // units per row block: head groups x request groups
+  int groups;   // > 0: grouped schedule with this many groups of `per` CTAs (one wave)
+  uint32_t* progress;  // [gridDim.x] pages consumed by each CTA's mixers (workspace, zeroed)
   WsHeader* ws;
 };
 
@@ -110,6 +115,28 @@ __device__ __forceinline__ Unit decode(const Params& p, int k) {
     u.Jmax = u.I1 >= 0 ? u.I1 : u.I0;
   }
   return u;
+}
+
+// The units of this CTA, longest first.  Grouped schedule (when a whole wave of `per` CTAs per
+// group fits the grid): the CTAs of group g each own one (head group, request group) and walk
+// the same row blocks n_rb - 1 - g - groups * t together, so the 16 or so CTAs that read a row
+// block's map tiles read them at about the same time and the tiles are fetched from DRAM once and
+// served from L2 to the others.  Otherwise: unit k = blockIdx.x + t * gridDim.x.
+__device__ __forceinline__ int units_of_cta(const Params& p) {
+  if (p.groups > 0) {
+    const int g = blockIdx.x / p.per;
+    return g < p.n_rb ? (p.n_rb - 1 - g) / p.groups + 1 : 0;
+  }
+  return (int)blockIdx.x < p.n_units ? (p.n_units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+}
+__device__ __forceinline__ Unit unit_at(const Params& p, int t) {
+  if (p.groups > 0) {
+    const int g = blockIdx.x / p.per, m = blockIdx.x % p.per;
+    const int rb = p.n_rb - 1 - (g + p.groups * t);
+    // (rb, hg, rg) -> the index decode() maps back to the same unit
+    return decode(p, (p.n_rb - 1 - rb) * p.per + m);
+  }
+  return decode(p, (int)blockIdx.x + t * (int)gridDim.x);
 }
 
 // Warp-collective: bit s set iff sender head s kept key block J in query block I.
@@ -192,6 +219,30 @@ __device__ void planner(Smem& s, const Params& p) {
     if (lane == 0) mbar_arrive(&s.plan_full[np % kPages]);
     ++np;
   };
+  // Keep the CTAs of a schedule group together (they read the same map tiles, which then come
+  // from DRAM once): hold page np back while the slowest member has consumed fewer than
+  // np - kPages - kPaceSlack pages.  A hint only: after kPaceNs it goes ahead regardless, so a
+  // member that is not resident (or finished) never blocks the others.
+  auto pace = [&]() {
+    if (p.groups <= 0 || p.per <= 1 || np <= (uint32_t)(kPages + kPaceSlack)) return;
+    const uint32_t need = np - (uint32_t)(kPages + kPaceSlack);
+    const int base = (int)(blockIdx.x / p.per) * p.per;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+      uint32_t lo = 0xffffffffu;
+      for (int m = lane; m < p.per; m += 32) {
+        const uint32_t v = ld_relaxed_gpu(p.progress + base + m);
+        lo = v < lo ? v : lo;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const uint32_t w = __shfl_xor_sync(0xffffffffu, lo, o);
+        lo = w < lo ? w : lo;
+      }
+      if (lo >= need || globaltimer_ns() - t0 > kPaceNs) break;
+      __nanosleep(256);
+    }
+  };
   auto marker = [&](uint32_t flags) {
     Page* pg = claim();
     if (!ok) return;
@@ -202,8 +253,9 @@ __device__ void planner(Smem& s, const Params& p) {
     }
     publish();
   };
-  for (int k = blockIdx.x; k < p.n_units && ok; k += gridDim.x) {
-    const Unit u = decode(p, k);
+  const int nu = units_of_cta(p);
+  for (int t = 0; t < nu && ok; ++t) {
+    const Unit u = unit_at(p, t);
     // lane l tracks sender heads l and l + 32, for the unit's one or two query blocks
     RowCursor cur[2][2];
     float wv[2][kAcc];
@@ -235,6 +287,7 @@ __device__ void planner(Smem& s, const Params& p) {
       const uint64_t uni = m0 | m1;
       if (uni != 0) {
         for (int h = 0; h < nparts && ok; ++h) {
+          pace();
           Page* pg = claim();
           if (!ok) break;
           // every lane writes the entries of its own sender heads, at their rank in the union
@@ -289,13 +342,14 @@ __device__ void planner(Smem& s, const Params& p) {
 // ------------------------------------------------------------------------------------------------
 // Walks the sub-steps (unit, key block J, 64-key panel h) of this CTA in order.  Warp-collective.
 struct SubWalker {
-  int k, J, h;
+  int t, nu, J, h;
   Unit u;
   bool live;
   __device__ __forceinline__ void start(const Params& p) {
-    k = blockIdx.x;
-    live = k < p.n_units;
-    if (live) u = decode(p, k);
+    t = 0;
+    nu = units_of_cta(p);
+    live = t < nu;
+    if (live) u = unit_at(p, t);
     J = 0;
     h = -1;
   }
@@ -317,9 +371,9 @@ struct SubWalker {
           return true;
         }
       }
-      k += gridDim.x;
-      live = k < p.n_units;
-      if (live) u = decode(p, k);
+      ++t;
+      live = t < nu;
+      if (live) u = unit_at(p, t);
       J = 0;
     }
     return false;
@@ -359,8 +413,9 @@ __device__ void mma_issuer(Smem& s, const Params& p, const CUtensorMap* tmap_v) 
     if (lane == 0) issue_v<G>(s, p, tmap_v, vw.u, vw.J * p.B + 64 * vw.h);
     ++nv;
   }
-  for (int k = blockIdx.x; k < p.n_units && ok; k += gridDim.x, ++nunit) {
-    const Unit u = decode(p, k);
+  const int nu = units_of_cta(p);
+  for (; nunit < nu && ok; ++nunit) {
+    const Unit u = unit_at(p, nunit);
     if (lane == 0 && nunit > 0 && !mbar_wait_sleep(&s.o_empty, (nunit - 1) & 1, &s.abort, kTimeoutNs, 64)) {
       fail(s, p, 0x201);
       ok = false;
@@ -480,7 +535,10 @@ __device__ void mixers(Smem& s, const Params& p) {
   };
   auto release_page = [&](uint32_t pg) {
     __syncwarp();
-    if (lane == 0) mbar_arrive(&s.plan_empty[pg % kPages]);
+    if (lane == 0) {
+      mbar_arrive(&s.plan_empty[pg % kPages]);
+      if (warp == 0) st_relaxed_gpu(p.progress + blockIdx.x, pg + 1);
+    }
   };
   // move the fetch cursor to the next page that lists panels (skipping markers); false on timeout
   auto fetch_seek = [&](uint32_t from) -> bool {
@@ -592,7 +650,7 @@ __device__ void mixers(Smem& s, const Params& p) {
   auto epilogue = [&](bool any) -> bool {
     if (!mbar_wait(&s.o_full, nunit & 1, &s.abort, kTimeoutNs)) return false;
     tc_fence_after();
-    const Unit u = decode(p, blockIdx.x + nunit * gridDim.x);
+    const Unit u = unit_at(p, nunit);
     const int row = 32 * tw + lane;
     const int i = u.rb * 128 + row;
 #pragma unroll 1
@@ -770,7 +828,9 @@ cudaError_t tc_retrieve(const RetrieveArgs& a) {
   p.n_rg = (a.n_req + p.R - 1) / p.R;
   p.n_rb = (a.map.L + 127) / 128;
   p.n_units = p.n_rb * p.n_hg * p.n_rg;
+  p.per = p.n_hg * p.n_rg;
   p.ws = a.ws;
+  p.progress = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(a.ws) + kWsHeaderBytes);
   // V viewed as rows of 128 bf16; rows are addressed from the request offset and head stride.
   // With strided requests the exact extent is known (rows past it read as zeros); with a device
   // offset table it is not, and the view spans the 32-bit row range.
@@ -783,7 +843,14 @@ cudaError_t tc_retrieve(const RetrieveArgs& a) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = p.n_units < sms ? p.n_units : sms;
+  int grid;
+  if (p.per <= sms && sms <= kMaxProgressCtas) {
+    p.groups = sms / p.per < p.n_rb ? sms / p.per : p.n_rb;
+    grid = p.groups * p.per;
+  } else {
+    p.groups = 0;
+    grid = p.n_units < sms ? p.n_units : sms;
+  }
   if (G == 4) return launch_g<4>(a, p, tm, grid, a.stream);
   if (G == 2) return launch_g<2>(a, p, tm, grid, a.stream);
   return launch_g<1>(a, p, tm, grid, a.stream);

@@ -65,6 +65,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// Relaxed gpu-scope accesses for counters that other CTAs poll.
+__device__ __forceinline__ void st_relaxed_gpu(uint32_t* ptr, uint32_t v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* ptr) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
+
 // As mbar_wait, for warps that mostly wait (producers, MMA issuers): sleeps between polls so the
 // warps that share its SM sub-partition keep the issue slots.
 __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, const volatile int* abort,
