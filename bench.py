@@ -194,11 +194,28 @@ def oracle_sample_time(spec, lay, units_I, rows, threads):
                          n_threads=threads)
     tr = time.perf_counter() - t0
     t_retrieve = tr * (L * (L + 1) / 2) / sum(i + 1 for i in rows)
-    desc = (f"{len(units)} compression units (h, I) with I in {sorted(set(int(i) for i in units_I))} and "
-            f"{len(rows)} retrieval rows {list(map(int, rows))} of the L={L} workload, "
+    desc = (f"{len(units)} compression units (h, I), I in [{min(units_I)}, {max(units_I)}], and "
+            f"{len(rows)} retrieval rows i in [{min(rows)}, {max(rows)}] of the L={L} workload, "
             f"extrapolated by per-unit work ((I+1) key blocks per unit, (i+1) keys per row); "
-            f"sample took {tc + tr:.1f} s")
+            f"sample took {tc + tr:.1f} s (compress {tc:.1f} s, retrieve {tr:.1f} s)")
     return t_compress + t_retrieve, desc, tc + tr
+
+
+def oracle_sample_calibrated(spec, lay, threads, target_s, rng):
+    """One bounded oracle sample of about `target_s` seconds: a calibration pass with one unit and
+    one row per thread, then units and rows (multiples of the thread count, so the pool stays full)
+    scaled to the target.  Returns (full-step seconds, description)."""
+    nqb = spec.L // spec.block
+
+    def draw(n):
+        return (rng.integers(nqb // 2, nqb, size=n).tolist(), rng.integers(spec.L // 2, spec.L, size=n).tolist())
+
+    u, r = draw(threads)
+    _, _, took = oracle_sample_time(spec, lay, u, r, threads)
+    reps = int(max(1, min(64, round(target_s / max(took, 1e-3)))))
+    u, r = draw(threads * reps)
+    t_full, desc, _ = oracle_sample_time(spec, lay, u, r, threads)
+    return t_full, desc
 
 
 def run_reference(args, spec, rank):
@@ -211,11 +228,12 @@ def run_reference(args, spec, rank):
     vals = []
     desc = ""
     for step in range(args.warmup + args.steps):
-        units_I = rng.integers(nqb // 2, nqb, size=threads).tolist()
-        rows = rng.integers(spec.L // 2, spec.L, size=max(1, threads // 4)).tolist()
-        t_full, desc, _ = oracle_sample_time(spec, lay, units_I, rows, threads)
-        if step >= args.warmup:
-            vals.append(spec.L / t_full)
+        if step < args.warmup:  # warm-up: one small pass (page-in, thread pool start)
+            u, r = rng.integers(nqb // 2, nqb, size=threads).tolist(), rng.integers(spec.L // 2, spec.L, size=threads).tolist()
+            oracle_sample_time(spec, lay, u, r, threads)
+            continue
+        t_full, desc = oracle_sample_calibrated(spec, lay, threads, 8.0, rng)
+        vals.append(spec.L / t_full)
     value = float(statistics.median(vals))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
@@ -421,10 +439,7 @@ def main():
     cpu = None
     if not args.no_cpu_baseline and world == 1 and rank == 0:
         threads = os.cpu_count() or 1
-        # one large unit and one late row per core keeps the cores evenly loaded
-        units_I = [nqb - 1 - 3 * k for k in range(threads)]
-        rows = [spec.L - 1 - 977 * k for k in range(threads)]
-        t_full, desc, took = oracle_sample_time(spec, lay, units_I, rows, threads)
+        t_full, desc = oracle_sample_calibrated(spec, lay, threads, 15.0, np.random.default_rng(11))
         cpu = {"value": spec.L / t_full, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc}
 
     if rank == 0:
