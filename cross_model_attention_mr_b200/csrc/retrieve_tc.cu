@@ -589,19 +589,19 @@ __device__ void mixers(Smem& s, const Params& p) {
   };
 
   constexpr int kW = 4 * kPieces;  // packed bf16 pairs per thread per panel
-  unsigned long long acc[G][kW];   // pairs of fp32 accumulators: columns (2e, 2e + 1) of the thread's chunks
+  float2 acc[G][kW];               // fp32 accumulators for columns (2e, 2e + 1) of the thread's chunks
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
-    for (int e = 0; e < kW; ++e) acc[g][e] = 0ull;
+    for (int e = 0; e < kW; ++e) acc[g][e] = make_float2(0.f, 0.f);
 
   // one entry: acc[g] += W[r_g, s] * (this thread's 16 values of the sender head's panel)
   auto mix_entry = [&](const Entry& E, uint32_t data) {
     const float4 wf = *reinterpret_cast<const float4*>(&E.w[0]);
     const float w[4] = {wf.x, wf.y, wf.z, wf.w};
-    unsigned long long w2[G];
+    float2 w2[G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) w2[g] = pack2(w[g], w[g]);
+    for (int g = 0; g < G; ++g) w2[g] = make_float2(w[g], w[g]);
 #pragma unroll
     for (int k = 0; k < kPieces; ++k) {
       const uint4 d = lds128(data + k * kPiece);
@@ -609,13 +609,11 @@ __device__ void mixers(Smem& s, const Params& p) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int c = 4 * k + e;
-        if constexpr (G == 4) {
-          mix_word4(acc[0][c], acc[1][c], acc[2][c], acc[3][c], wd[e], w2[0], w2[1], w2[2], w2[3]);
-        } else {
-          const unsigned long long v2 = pack2(__uint_as_float(wd[e] << 16), __uint_as_float(wd[e] & 0xffff0000u));
+        // bf16 pair -> fp32 pair: the low half is the lower column (measured: a shift here beats a
+        // byte permute, which loads the integer pipe with both halves)
+        const float2 v = make_float2(__uint_as_float(wd[e] << 16), __uint_as_float(wd[e] & 0xffff0000u));
 #pragma unroll
-          for (int g = 0; g < G; ++g) acc[g][c] = ffma2(w2[g], v2, acc[g][c]);
-        }
+        for (int g = 0; g < G; ++g) acc[g][c] = __ffma2_rn(w2[g], v, acc[g][c]);
       }
     }
   };
@@ -630,11 +628,10 @@ __device__ void mixers(Smem& s, const Params& p) {
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          float lo, hi;
-          unpack2(acc[g][4 * k + e], lo, hi);
-          const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);
+          const float2 a = acc[g][4 * k + e];
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(a.x, a.y);
           pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
-          acc[g][4 * k + e] = 0ull;
+          acc[g][4 * k + e] = make_float2(0.f, 0.f);
         }
         char* xb = reinterpret_cast<char*>(&s.x[g][0]) + (rowb + 4 * k) * 128 + (lane & 7) * 16;
         *reinterpret_cast<uint4*>(xb) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
