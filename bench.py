@@ -218,6 +218,32 @@ def oracle_sample_calibrated(spec, lay, threads, target_s, rng):
     return t_full, desc
 
 
+# ------------------------------------------------------------------------------------------------
+# multi-rank host logic (one process per GPU; independent sequences, no data-path collective)
+# ------------------------------------------------------------------------------------------------
+def rank_spec(spec, rank: int):
+    """Rank r processes its own sequence: the same workload drawn from seed + 7919 r."""
+    if spec.seed is None or rank == 0:
+        return spec
+    from dataclasses import replace
+    return replace(spec, seed=spec.seed + 7919 * rank)
+
+
+def max_over_ranks(ms: float, dist, device) -> float:
+    """Slowest rank's time (the job is done when every rank is)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, L: int, ms: float) -> float:
+    """Whole-job throughput: every rank processed L tokens in the slowest rank's time."""
+    return world * L / (ms / 1e3)
+
+
 def run_reference(args, spec, rank):
     if rank != 0:
         return
@@ -286,9 +312,7 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local))
-    if spec.seed is not None and rank:
-        from dataclasses import replace
-        spec = replace(spec, seed=spec.seed + 7919 * rank)  # independent sequence per rank
+    spec = rank_spec(spec, rank)  # independent sequence per rank
 
     lay = draw_layers(spec)[0]
     bf = torch.bfloat16
@@ -351,11 +375,8 @@ def main():
     st_c, st_r = ws_c.sync_status(), ws_r.sync_status()
     if st_c or st_r:
         raise SystemExit(f"device status in the timed steps: compress={st_c} retrieve={st_r}")
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * spec.L / (ms / 1e3)
+    ms = max_over_ranks(ms, dist, "cuda")
+    value = job_tokens_per_s(world, spec.L, ms)
 
     # ---- roofline of the dominant kernel ----
     pk, pk_src = peaks()
@@ -407,11 +428,8 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         ems = e0.elapsed_time(e1) / n_e2e
-        if dist is not None:
-            t = torch.tensor([ems], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * spec.L / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+        ems = max_over_ranks(ems, dist, "cuda")
+        e2e = {"value": job_tokens_per_s(world, spec.L, ems), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": ems}
 
     # ---- what the receiver would otherwise run: dense causal attention of its 64 heads ----
