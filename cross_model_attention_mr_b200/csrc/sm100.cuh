@@ -105,14 +105,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// Contiguous bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16).
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
-
 // Bring `bytes` (multiple of 16) of global memory into L2 without touching shared memory.
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
@@ -174,10 +166,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 
-__device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t& r) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
-}
-
 __device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
 }
@@ -196,34 +184,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
-}
-
-// Packed fp32 pairs: d = a * b + c on both halves of a 64-bit register pair (one instruction).
-__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b, unsigned long long c) {
-  unsigned long long d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-// acc[g] += w2[g] * (lo, hi) for the two bf16 values packed in `x` (low half = lower column),
-// g = 0..3: one word unpacked once, pairs formed in registers (no moves), four FFMA2.
-__device__ __forceinline__ void mix_word4(unsigned long long& a0, unsigned long long& a1, unsigned long long& a2,
-                                          unsigned long long& a3, uint32_t x, unsigned long long w0,
-                                          unsigned long long w1, unsigned long long w2, unsigned long long w3) {
-  asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 v;\n\t"
-      "shl.b32 lo, %4, 16;\n\tand.b32 hi, %4, 0xffff0000;\n\tmov.b64 v, {lo, hi};\n\t"
-      "fma.rn.f32x2 %0, %5, v, %0;\n\tfma.rn.f32x2 %1, %6, v, %1;\n\t"
-      "fma.rn.f32x2 %2, %7, v, %2;\n\tfma.rn.f32x2 %3, %8, v, %3;\n\t}"
-      : "+l"(a0), "+l"(a1), "+l"(a2), "+l"(a3)
-      : "r"(x), "l"(w0), "l"(w1), "l"(w2), "l"(w3));
-}
-
-__device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
-  unsigned long long d;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
-  return d;
-}
-__device__ __forceinline__ void unpack2(unsigned long long v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
 
 // 2^x on the multi-function unit (relative error about 2^-22; flushes subnormal results to 0).

@@ -116,6 +116,53 @@ def test_one_or_two_sender_heads_long_units(mr, n, H_s, H_r):
     compare_retrieve(spec, lay, m, O, np.arange(0, spec.L, 7))
 
 
+def _retrieve_requests(mr, spec, lay, V_req):
+    """Compress once, retrieve n_req strided value sets [n_req][H_r][L][d_v] in one launch."""
+    Q, K = dev(lay.Q, spec.dtype), dev(lay.K, spec.dtype)
+    m = mr.compress(Q, K, p32(spec.p), spec.block, bias=mr.Bias.from_spec(lay.bias), scale=spec.scale)
+    assert m.ws.sync_status() == mr.MR_OK
+    n_req = V_req.shape[0]
+    ws_r = mr.Workspace(mr.retrieve_workspace_bytes(m, spec.H_r, spec.d_v, n_req))
+    O = mr.retrieve(m, torch.from_numpy(lay.W).cuda(), dev(V_req, spec.dtype), ws=ws_r)
+    torch.cuda.synchronize()
+    check_retrieve_status(mr, ws_r)
+    return m, O
+
+
+@pytest.mark.parametrize("n_req", [2, 4, 5])
+def test_request_groups_strided_values(mr, n_req):
+    """2 requests: 2 heads x 2 requests per CTA; 4 or 5: 1 head x 4 requests (the 5th request in
+    a partial request group).  Values strided per request."""
+    from cross_model_attention_mr_b200.workloads import Layer
+    spec = shrink(config(2), L=768, H_s=4, H_r=3)
+    lay = draw_layers(spec)[0]
+    rng = np.random.default_rng(77 + n_req)
+    V_req = rng.standard_normal((n_req, spec.H_r, spec.L, spec.d_v), dtype=np.float32)
+    V_req = V_req.astype(np.float32)
+    from cross_model_attention_mr_b200.workloads import round_to_bf16
+    V_req = round_to_bf16(V_req)
+    m, O = _retrieve_requests(mr, spec, lay, V_req)
+    rows = np.array([0, 1, 63, 64, 129, 383, 500, 767])
+    for q in range(n_req):
+        lq = Layer(Q=lay.Q, K=lay.K, V=np.ascontiguousarray(V_req[q]), W=lay.W, bias=lay.bias)
+        compare_retrieve(spec, lq, m, O[q:q + 1], rows)
+
+
+def test_ungrouped_schedule_many_receiver_heads(mr):
+    """160 receiver heads x 4 requests: one row block needs 160 CTAs, more than the SMs, so the
+    retrieval falls back to the ungrouped schedule."""
+    from cross_model_attention_mr_b200.workloads import Layer, round_to_bf16
+    spec = shrink(config(4), L=512, H_s=2, H_r=160)
+    lay = draw_layers(spec)[0]
+    rng = np.random.default_rng(91)
+    V_req = round_to_bf16(rng.standard_normal((4, spec.H_r, spec.L, spec.d_v), dtype=np.float32))
+    m, O = _retrieve_requests(mr, spec, lay, V_req)
+    rows = np.array([0, 127, 128, 300, 511])
+    for q in (0, 3):
+        lq = Layer(Q=lay.Q, K=lay.K, V=np.ascontiguousarray(V_req[q]), W=lay.W, bias=lay.bias)
+        compare_retrieve(spec, lq, m, O[q:q + 1], rows)
+
+
 def test_capacity_overflow_is_reported(mr):
     spec = shrink(config(2), L=512, H_s=2, H_r=2)
     lay = draw_layers(spec)[0]
