@@ -850,6 +850,7 @@ cudaError_t tc_retrieve(const RetrieveArgs& a) {
   } else {
     p.groups = 0;
     grid = p.n_units < sms ? p.n_units : sms;
+    if (grid > kMaxProgressCtas) grid = kMaxProgressCtas;  // one progress counter per CTA
   }
   if (G == 4) return launch_g<4>(a, p, tm, grid, a.stream);
   if (G == 2) return launch_g<2>(a, p, tm, grid, a.stream);
