@@ -239,6 +239,17 @@ def max_over_ranks(ms: float, dist, device) -> float:
     return float(t.item())
 
 
+def all_ranks_ok(ok: bool, dist, device) -> bool:
+    """Every rank learns whether all ranks are fine, so an error path takes the same collective
+    steps everywhere (no rank is left waiting in a later collective)."""
+    if dist is None:
+        return ok
+    import torch
+    t = torch.tensor([1 if ok else 0], dtype=torch.int32, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MIN)
+    return bool(t.item())
+
+
 def job_tokens_per_s(world: int, L: int, ms: float) -> float:
     """Whole-job throughput: every rank processed L tokens in the slowest rank's time."""
     return world * L / (ms / 1e3)
@@ -310,7 +321,7 @@ def main():
     if world > 1:
         import datetime
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     spec = rank_spec(spec, rank)  # independent sequence per rank
 
@@ -344,8 +355,8 @@ def main():
         step()
     torch.cuda.synchronize()
     st_c, st_r = ws_c.sync_status(), ws_r.sync_status()
-    if st_c or st_r:
-        raise SystemExit(f"device status compress={st_c} retrieve={st_r}")
+    if not all_ranks_ok(not (st_c or st_r), dist, "cuda"):
+        raise SystemExit(f"device status (this rank) compress={st_c} retrieve={st_r}")
     nnz = m.nnz_host()
     kept = m.kept_bits_host()
     nqb = spec.L // spec.block
@@ -373,8 +384,8 @@ def main():
     launches = mr.kernel_launches() - launches0
     ms = ev0.elapsed_time(ev1) / args.steps
     st_c, st_r = ws_c.sync_status(), ws_r.sync_status()
-    if st_c or st_r:
-        raise SystemExit(f"device status in the timed steps: compress={st_c} retrieve={st_r}")
+    if not all_ranks_ok(not (st_c or st_r), dist, "cuda"):
+        raise SystemExit(f"device status in the timed steps (this rank): compress={st_c} retrieve={st_r}")
     ms = max_over_ranks(ms, dist, "cuda")
     value = job_tokens_per_s(world, spec.L, ms)
 
@@ -449,8 +460,8 @@ def main():
         e1.record(s_out)
         torch.cuda.synchronize()
         st_c, st_r = ws_c.sync_status(), ws_r.sync_status()
-        if st_c or st_r:
-            raise SystemExit(f"device status in the end-to-end steps: compress={st_c} retrieve={st_r}")
+        if not all_ranks_ok(not (st_c or st_r), dist, "cuda"):
+            raise SystemExit(f"device status in the end-to-end steps (this rank): compress={st_c} retrieve={st_r}")
         ems = e0.elapsed_time(e1) / n_e2e
         ems = max_over_ranks(ems, dist, "cuda")
         e2e = {"value": job_tokens_per_s(world, spec.L, ems), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),

@@ -39,7 +39,9 @@ def _rank_main(rank, world, port, out):
         dist.all_gather(sigs, sig)
         ms = bench.max_over_ranks(10.0 + 5.0 * rank, dist, "cpu")
         value = bench.job_tokens_per_s(world, spec.L, ms)
-        out[rank] = (spec.seed, [float(x.item()) for x in sigs], ms, value)
+        all_fine = bench.all_ranks_ok(True, dist, "cpu")
+        one_failed = bench.all_ranks_ok(rank != 1, dist, "cpu")  # rank 1 reports a device error
+        out[rank] = (spec.seed, [float(x.item()) for x in sigs], ms, value, all_fine, one_failed)
     finally:
         dist.destroy_process_group()
 
@@ -54,9 +56,10 @@ def test_two_gloo_ranks_independent_sequences_and_max_time():
     sigs = out[0][1]
     assert sigs == out[1][1] and sigs[0] != sigs[1]  # different sequences, seen alike by both ranks
     for r in range(world):
-        _, _, ms, value = out[r]
+        _, _, ms, value, all_fine, one_failed = out[r]
         assert ms == pytest.approx(15.0)  # the slowest rank's time on every rank
         assert value == pytest.approx(world * 256 / 15e-3)
+        assert all_fine and not one_failed  # every rank takes the error path together
 
 
 def test_single_rank_helpers_without_a_process_group():
@@ -67,3 +70,4 @@ def test_single_rank_helpers_without_a_process_group():
     assert bench.rank_spec(spec, 0) is spec
     assert bench.max_over_ranks(12.5, None, "cpu") == 12.5
     assert bench.job_tokens_per_s(1, 32768, 100.0) == pytest.approx(327680.0)
+    assert bench.all_ranks_ok(False, None, "cpu") is False
