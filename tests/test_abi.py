@@ -97,6 +97,13 @@ def test_retrieve_and_dense_reject_bad_arguments(mr):
     assert r(n=0) == mr.MR_ERR_INVALID_ARG
     assert r(hs=10) == mr.MR_ERR_INVALID_ARG
     assert r(dt=1) == mr.MR_ERR_UNSUPPORTED
+    # the workspace holds the status header and one progress counter per CTA (up to 1024)
+    need = lib.mr_retrieve_workspace_bytes(ctypes.byref(b), 5, 64, 1)
+    assert need == 256 + 1024 * 4
+    ok_args = lambda wsb: lib.mr_retrieve(ctypes.byref(b), fake, 5, fake, fake, 0, 64, 1, None, 0, 512 * 64,
+                                          fake, wsb, None)
+    assert ok_args(need - 1) == mr.MR_ERR_INVALID_ARG  # rejected before anything is launched
+    assert ok_args(256) == mr.MR_ERR_INVALID_ARG
     d = lambda **kw: lib.mr_dense_ref(fake, fake, fake, fake, kw.get("dt", 0), 4, kw.get("d", 64), 64,
                                       kw.get("cu", fake), fake, None, 2, 100, 100, 0.125, None, fake, 4096, None)
     assert d(cu=None) == mr.MR_ERR_INVALID_ARG
