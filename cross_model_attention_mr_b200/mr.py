@@ -191,6 +191,49 @@ class Map:
         return out[:n]
 
 
+# ------------------------------------------------------------------------------------------------
+# Moving a compressed map to another rank (MapFlow section 5.3: the sender's compressed maps are
+# shipped to the receiver instance, which then runs the fused retrieval locally).
+# torch.distributed point-to-point: NCCL between GPUs, gloo between CPU ranks.
+# ------------------------------------------------------------------------------------------------
+def _map_arrays(m: "Map", n_stored: int):
+    arrays = [m.row_ptr, m.kept_bits, m.kept_mass]
+    if n_stored > 0:
+        # bf16 travels as its bit pattern, so every backend moves it unchanged
+        vals = m.vals[:n_stored]
+        arrays += [m.col_idx[:n_stored], vals.view(torch.int16) if vals.dtype == torch.bfloat16 else vals]
+    return arrays
+
+
+def send_map(m: "Map", dst: int, group=None) -> None:
+    """Send the arrays the retrieval reads: row pointers, kept bits and masses, and the column
+    indices and values of the stored tiles (min(kept tiles, capacity) of them)."""
+    import torch.distributed as dist
+    nnz = int(m.nnz.item())
+    n = min(nnz, m.capacity)
+    hdr = torch.tensor([m.H_s, m.L, m.block, m.dtype, nnz, n], dtype=torch.int64, device=m.row_ptr.device)
+    dist.send(hdr, dst, group=group)
+    for t in _map_arrays(m, n):
+        dist.send(t.contiguous(), dst, group=group)
+
+
+def recv_map(src: int, device="cuda", group=None) -> "Map":
+    """Receive a map sent by send_map into a new Map on `device` whose capacity is the number of
+    stored tiles; the kept-tile count is the sender's (tiles past the sender's capacity stay
+    unstored, as they were)."""
+    import torch.distributed as dist
+    hdr = torch.empty(6, dtype=torch.int64, device=device)
+    dist.recv(hdr, src, group=group)
+    H_s, L, block, dtype, nnz, n = (int(x) for x in hdr.tolist())
+    m = Map(H_s, L, block, dtype, max(1, n), device)
+    m.capacity = n
+    m.c.capacity_tiles = n
+    for t in _map_arrays(m, n):
+        dist.recv(t, src, group=group)
+    m.nnz.fill_(nnz)
+    return m
+
+
 def max_tiles(H_s: int, L: int, block: int) -> int:
     return int(LIB.mr_bsr_max_tiles(H_s, L, block))
 
