@@ -30,7 +30,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from cross_model_attention_mr_b200.workloads import config, draw_layers, shrink  # noqa: E402
+from cross_model_attention_mr_b200.workloads import config, draw_batch, draw_layers, shrink  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "prefill tokens/s for compress+retrieve at L=32K; % TC peak and % HBM peak"
@@ -286,6 +286,158 @@ def run_reference(args, spec, rank):
 
 
 # ------------------------------------------------------------------------------------------------
+# measurement lines for the other workloads (one GPU; the headline line is the default, config 4)
+# ------------------------------------------------------------------------------------------------
+CONFIG_METRIC = {
+    2: "prefill tokens/s for compress+retrieve, 1 layer, L=4K, 32 -> 40 heads, block 64",
+    3: "prefill tokens/s for compress+retrieve summed over 28 layers, L=8K, 32 -> 28 heads, block 64",
+    5: "prefill tokens/s: shared 4K prefix compressed once, retrieval for 16 requests, dense causal "
+       "rows for their 512-2048-token suffixes",
+}
+
+
+def config_tokens_per_step(spec, suffixes=None) -> int:
+    """Tokens one step processes: the sequence, or (config 5) every request's prefix + suffix."""
+    if suffixes is None:
+        return spec.L
+    return int(sum(spec.L + int(x) for x in suffixes))
+
+
+def run_config_line(args, spec, n):
+    """One timed measurement line for workload n in {2, 3, 5} on one GPU (same JSON contract;
+    end-to-end and CPU baseline are reported for the headline workload only)."""
+    import torch
+    from cross_model_attention_mr_b200 import mr
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    bf = torch.bfloat16
+    to_dev = lambda x: torch.from_numpy(x).to(bf).cuda().contiguous()  # noqa: E731
+    p = float(np.float32(spec.p))
+    cap = mr.max_tiles(spec.H_s, spec.L, spec.block)
+    m = mr.Map(spec.H_s, spec.L, spec.block, mr.MR_BF16, cap, "cuda")
+    ws_c = mr.Workspace(mr.compress_workspace_bytes(spec.H_s, spec.L, spec.d, spec.block))
+    suffixes = None
+    nqb = spec.L // spec.block
+    if n in (2, 3):
+        layers = draw_layers(spec)
+        dev = [(to_dev(l.Q), to_dev(l.K), to_dev(l.V), torch.from_numpy(l.W).cuda(), mr.Bias.from_spec(l.bias))
+               for l in layers]
+        ws_r = mr.Workspace(mr.retrieve_workspace_bytes(m, spec.H_r, spec.d_v, 1))
+        O = torch.empty((1, spec.H_r, spec.L, spec.d_v), dtype=bf, device="cuda")
+        wss = [ws_c, ws_r]
+
+        def step():
+            for Q, K, V, W, bias in dev:
+                mr.compress(Q, K, p, spec.block, bias=bias, scale=spec.scale, out=m, ws=ws_c, stream=stream)
+                mr.retrieve(m, W, V, out=O, ws=ws_r, stream=stream)
+
+        def per_layer_maps():
+            out = []
+            for Q, K, V, W, bias in dev:
+                mr.compress(Q, K, p, spec.block, bias=bias, scale=spec.scale, out=m, ws=ws_c, stream=stream)
+                out.append((m.nnz_host(), int(np.any(m.kept_bits_host(), axis=0).sum())))
+            return out
+    else:
+        b = draw_batch(spec)
+        P, R = spec.L, spec.n_req
+        suffixes = [r.suffix for r in b.requests]
+        lens_k = [P + x for x in suffixes]
+        cu_k = np.concatenate([[0], np.cumsum(lens_k)]).astype(np.int32)
+        cu_q = np.concatenate([[0], np.cumsum(suffixes)]).astype(np.int32)
+        Qs, Ks = to_dev(b.Qs), to_dev(b.Ks)
+        W = torch.from_numpy(b.W).cuda()
+        bias_s = mr.Bias.from_spec(b.bias)
+        bias_r = mr.Bias(b.bias.sink_len, b.bias.sink_bias, b.bias.window, b.bias.window_bias)
+        Vp = to_dev(np.concatenate([r.V for r in b.requests], axis=1))        # [H_r][total_k][d_v]
+        Kp = to_dev(np.concatenate([r.K for r in b.requests], axis=1))        # [H_r][total_k][d]
+        Qsuf = to_dev(np.concatenate([r.Q[:, P:] for r in b.requests], axis=1))  # [H_r][total_q][d]
+        off = torch.tensor(cu_k[:-1].astype(np.int64) * spec.d_v, dtype=torch.int64, device="cuda")
+        cu_q_d, cu_k_d = torch.from_numpy(cu_q).cuda(), torch.from_numpy(cu_k).cuda()
+        q_off = torch.full((R,), P, dtype=torch.int32, device="cuda")
+        ws_r = mr.Workspace(mr.retrieve_workspace_bytes(m, spec.H_r, spec.d_v, R))
+        ws_d = mr.Workspace(mr.LIB.mr_dense_ref_workspace_bytes(R))
+        O_ret = torch.empty((R, spec.H_r, P, spec.d_v), dtype=bf, device="cuda")
+        O_suf = torch.empty((spec.H_r, int(cu_q[-1]), spec.d_v), dtype=bf, device="cuda")
+        wss = [ws_c, ws_r, ws_d]
+
+        def step():
+            mr.compress(Qs, Ks, p, spec.block, bias=bias_s, scale=spec.scale, out=m, ws=ws_c, stream=stream)
+            mr.retrieve(m, W, Vp, out=O_ret, v_req_off=off, v_head_stride=int(cu_k[-1]) * spec.d_v, n_req=R,
+                        ws=ws_r, stream=stream)
+            mr.dense_ref(Qsuf, Kp, Vp, cu_q_d, cu_k_d, q_off, int(cu_q[-1]), int(cu_k[-1]), bias=bias_r,
+                         scale=spec.scale, out=O_suf, ws=ws_d, stream=stream)
+
+        def per_layer_maps():
+            mr.compress(Qs, Ks, p, spec.block, bias=bias_s, scale=spec.scale, out=m, ws=ws_c, stream=stream)
+            return [(m.nnz_host(), int(np.any(m.kept_bits_host(), axis=0).sum()))]
+
+    maps = per_layer_maps()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if any(w.sync_status() for w in wss):
+        raise SystemExit(f"device status after warm-up: {[w.sync_status() for w in wss]}")
+    sampler = ClockSampler(gpu_index_for(0))
+    sampler.start()
+    time.sleep(0.3)
+    launches0 = mr.kernel_launches()
+    mr.profile_enable(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    prof = mr.profile_read()
+    mr.profile_enable(False)
+    launches = mr.kernel_launches() - launches0
+    if any(w.sync_status() for w in wss):
+        raise SystemExit(f"device status in the timed steps: {[w.sync_status() for w in wss]}")
+    ms = ev0.elapsed_time(ev1) / args.steps
+    tokens = config_tokens_per_step(spec, suffixes)
+    n_req = spec.n_req if n == 5 else 1
+    per_layer = [algorithmic(spec, nnz, un, n_req) for nnz, un in maps]
+    work = {k: sum(w[k] for w in per_layer) / len(per_layer) for k in per_layer[0]}  # per launch, layer mean
+    pk, pk_src = peaks()
+    dname, (dms, dcnt) = max(prof.items(), key=lambda kv: kv[1][0])
+    bound, amount, _ = kernel_work(dname, work)
+    roofline = None
+    if bound is not None:
+        avg_s = dms / dcnt / 1e3
+        if bound == "hbm":
+            achieved, peak, runit, kind = amount / avg_s / 1e9, float(pk["hbm_gbs"]), "GB/s", "copy"
+        elif bound == "alu":
+            sms = torch.cuda.get_device_properties(0).multi_processor_count
+            achieved, runit, kind = amount / avg_s / 1e12, "TFLOP/s", "fp32 FMA"
+            peak, pk_src = sms * 128 * 2 * float(pk.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12, "derived"
+        else:
+            achieved, runit, kind = amount / avg_s / 1e12, "TFLOP/s", "sustained"
+            peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+        roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": runit, "frac": achieved / peak,
+                    "traffic": None, "kernel": dname, "peak_source": pk_src, "peak_kind": kind}
+    total = sum(v[0] for v in prof.values())
+    stages = {k: {"ms_per_launch": v[0] / v[1], "launches": v[1], "share": v[0] / total} for k, v in prof.items()}
+    nnz_all = sum(x[0] for x in maps)
+    tiles_all = len(maps) * spec.H_s * nqb * (nqb + 1) / 2
+    line = {
+        "metric": CONFIG_METRIC[n], "value": tokens / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": spec.name, "L": spec.L, "H_s": spec.H_s, "H_r": spec.H_r, "d": spec.d,
+                   "block": spec.block, "p": spec.p, "layers": len(maps) if n == 3 else 1,
+                   "requests": n_req, "tokens_per_step": tokens,
+                   "l2": "inputs larger than L2 (maps %.2f GB per step)" % (nnz_all * spec.block ** 2 * 2 / 1e9),
+                   "parallelism": "replicas1"},
+        "gpu_launches": int(launches), "clocks": clocks, "roofline": roofline,
+        "cpu_baseline": None, "e2e": None, "stages": stages,
+        "map": {"nnz_tiles": nnz_all, "kept_fraction": nnz_all / tiles_all,
+                "union_fraction": sum(x[1] for x in maps) / (len(maps) * nqb * (nqb + 1) / 2)},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------------
 # native arm
 # ------------------------------------------------------------------------------------------------
 def main():
@@ -299,15 +451,23 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--L", type=int, default=None,
                     help="shorter sequence of the same workload shape (profiling captures); default 32768")
+    ap.add_argument("--config", type=int, default=4, choices=[2, 3, 4, 5],
+                    help="workload: 4 = the headline line (default); 2, 3, 5 = one-GPU measurement lines")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    spec = config(4)
+    spec = config(args.config)
     if args.L is not None and args.L != spec.L:
-        spec = shrink(spec, L=args.L, name=spec.name.replace("L32768", f"L{args.L}"))
+        name = spec.name.replace("L32768", f"L{args.L}") if "L32768" in spec.name else f"{spec.name}_at_L{args.L}"
+        spec = shrink(spec, L=args.L, name=name)
+    if args.config != 4 and args.impl != "reference":
+        if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+            raise SystemExit("--config 2/3/5 lines are one-GPU measurements")
+        run_config_line(args, spec, args.config)
+        return
 
     if args.impl == "reference":
         run_reference(args, spec, rank)

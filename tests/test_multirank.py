@@ -71,6 +71,9 @@ def test_single_rank_helpers_without_a_process_group():
     assert bench.max_over_ranks(12.5, None, "cpu") == 12.5
     assert bench.job_tokens_per_s(1, 32768, 100.0) == pytest.approx(327680.0)
     assert bench.all_ranks_ok(False, None, "cpu") is False
+    # the other workloads' lines: tokens per step (config 5: every request's prefix and suffix)
+    assert bench.config_tokens_per_step(config(2)) == 4096
+    assert bench.config_tokens_per_step(config(5), [512, 2048, 1000]) == 3 * 4096 + 3560
 
 
 def _synthetic_map(mr, nnz, capacity, seed):
