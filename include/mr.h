@@ -142,6 +142,9 @@ int64_t mr_bsr_max_tiles(int H_s, int L, int block);
  *   ws     workspace of at least mr_compress_workspace_bytes(H_s, L, d, block) bytes.
  * Supported: d in {64, 128}; block in {64, 128}; L a positive multiple of block with
  * L / block <= 256; H_s <= 64.  MR_BF16 maps use bf16 vals; MR_F32 maps use fp32 vals.
+ * bf16 with d = 128 (and per-key-block biases, if any, on multiples of 32 keys) runs on the
+ * tensor-core kernels; other shapes on the CUDA-core kernels.  Either way vals hold the tiles in
+ * the 128-byte-panel layout described at mr_bsr.
  * If the map needs more than capacity_tiles tiles, the status word records MR_ERR_CAPACITY and
  * no tile at or beyond capacity_tiles is written (nnz still reports the full count).
  */
@@ -181,7 +184,12 @@ mr_status mr_compress_noalloc(const void* Q, const void* K, mr_dtype dt, int H_s
                               float scale, float p, const mr_logit_bias* bias, mr_bsr* out,
                               void* stream);
 
-/* Workspace bytes mr_retrieve needs (device memory, 256-byte aligned). */
+/*
+ * Workspace bytes mr_retrieve needs (device memory, 256-byte aligned): the status header and one
+ * progress counter per CTA, which the CTAs of a schedule group read to stay together (the ones
+ * that read the same map tiles then find them in L2).  mr_retrieve zeroes it before its launch;
+ * calls that overlap on the GPU need separate workspaces.
+ */
 size_t mr_retrieve_workspace_bytes(const mr_bsr* map, int H_r, int d_v, int n_req);
 
 /*
@@ -197,7 +205,10 @@ size_t mr_retrieve_workspace_bytes(const mr_bsr* map, int H_r, int d_v, int n_re
  *          v_off(q) = v_req_off[q] (device int64 array) or q * v_req_stride when v_req_off is NULL
  *   O      output in dtype dt: element (q, r, i, c) at O + q * H_r * L * d_v + (r * L + i) * d_v + c
  *   ws     workspace of at least mr_retrieve_workspace_bytes(map, H_r, d_v, n_req) bytes
- * Supported: d_v in {64, 128}; H_r <= 256.
+ * Supported: d_v in {64, 128}; H_r <= 256.  bf16 maps with d_v = 128, block 64 or 128 and
+ * H_s <= 64 run on the tensor-core kernel; other shapes on the CUDA-core kernel.
+ * Tiles a map could not store (capacity overflow at compression) contribute nothing and set
+ * MR_ERR_CAPACITY in the status word.
  */
 mr_status mr_retrieve(const mr_bsr* map, const float* W, int H_r, const void* V, void* O,
                       mr_dtype dt, int d_v, int n_req, const int64_t* v_req_off,
