@@ -1,7 +1,8 @@
 """Python binding of libmr (argument marshalling only; every step of the path runs in libmr's kernels).
 
 The names follow the C-ABI in ``include/mr.h``: ``compress`` -> ``mr_compress``, ``retrieve`` ->
-``mr_retrieve``, ``dense_ref`` -> ``mr_dense_ref``.  PyTorch is used for device memory and streams.
+``mr_retrieve``, ``dense_ref`` -> ``mr_dense_ref``.  PyTorch is used for device memory and streams;
+``send_map`` / ``recv_map`` move a compressed map between ranks with torch.distributed.
 Importing this module loads ``libmr.so`` and raises ``ImportError`` if it has not been built:
 there is no fallback implementation.
 """
