@@ -11,6 +11,7 @@ this module only marshals numpy arrays.  Each wrapper names the passage it follo
                         ("Accelerating Cross-Model LLM Inference via Attention Map Reuse", s4, s5.2)
   * ``select``       -- the top-p rule on one row of block masses (same sections)
   * ``tile_probs``   -- softmax probabilities of one map tile (s2.1)
+  * ``row_block_probs`` -- the same softmax rows for whole query blocks (s2.1)
   * ``retrieve_rows``-- translated map times receiver values on given kept sets (s3.3, s5.4)
   * ``dense_rows``   -- exact causal attention ("AttnCache Guide", "The Quadratic Self-Attention Cost")
 """
@@ -55,13 +56,16 @@ def _load():
                                                                  ctypes.c_int, ctypes.c_int]
         lib.or_tile_probs.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, f64,
                                       ctypes.c_int] + bias_args + [ctypes.c_int] * 3 + [P]
+        lib.or_row_block_probs.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, f64,
+                                           ctypes.c_int] + bias_args + [P, ctypes.c_int, P, ctypes.c_int]
         lib.or_retrieve_rows.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, f64,
                                          ctypes.c_int] + bias_args + [
             P, P, ctypes.c_int, P, ctypes.c_int, i64, ctypes.c_int, P, ctypes.c_int, P,
             ctypes.c_int]
         lib.or_dense_rows.argtypes = [P, P, P] + [ctypes.c_int] * 5 + [i64, f64] + bias_args + [
             P, ctypes.c_int, P, ctypes.c_int]
-        for name in ("or_compress", "or_tile_probs", "or_retrieve_rows", "or_dense_rows"):
+        for name in ("or_compress", "or_tile_probs", "or_row_block_probs", "or_retrieve_rows",
+                     "or_dense_rows"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -129,6 +133,21 @@ def tile_probs(Q, K, sigma: float, B: int, h: int, I: int, J: int, bias=None) ->
                                int(J), _ptr(out))
     if rc:
         raise ValueError("oracle tile_probs rejected its arguments")
+    return out
+
+
+def row_block_probs(Q, K, sigma: float, B: int, units: Sequence[int], bias=None,
+                    n_threads: int = 0) -> np.ndarray:
+    """Softmax rows of whole query blocks: [len(units)][B][L] for units u = h*nQB + I (s2.1)."""
+    Q, K = _f32(Q), _f32(K)
+    H, L, d = Q.shape
+    u = np.ascontiguousarray(units, dtype=np.int32)
+    out = np.zeros((u.shape[0], B, L), np.float64)
+    ba, keep = _bias_args(bias)
+    rc = _load().or_row_block_probs(_ptr(Q), _ptr(K), H, L, d, float(sigma), int(B), *ba, _ptr(u),
+                                    int(u.shape[0]), _ptr(out), int(n_threads))
+    if rc:
+        raise ValueError("oracle row_block_probs rejected its arguments")
     return out
 
 

@@ -235,6 +235,40 @@ OR_EXPORT int or_tile_probs(const float* Q, const float* K, int H, int L, int d,
     return 0;
 }
 
+/* Probabilities of every row of query block I of head h over all L keys, for a list of units
+ * u = h * nQB + I: out[t][a][j] = A_h[I*B + a][j] for j <= I*B + a, else 0 ([MF] s2.1).  The rows are
+ * the same softmax rows as or_tile_probs; this form returns a whole row block at once (a slab of
+ * B x L) so that every stored tile of a unit can be checked without recomputing its rows.
+ *   out : [n_units][B][L] */
+OR_EXPORT int or_row_block_probs(const float* Q, const float* K, int H, int L, int d, double sigma,
+                                 int B, int32_t sink_len, double sink_bias, int32_t window,
+                                 double window_bias, const float* kb_bias, int32_t kb_block,
+                                 const int32_t* units, int n_units, double* out, int n_threads)
+{
+    if (B <= 0 || L % B) return 1;
+    const int nQB = L / B;
+    for (int t = 0; t < n_units; ++t)
+        if (units[t] < 0 || units[t] >= H * nQB) return 1;
+    or_bias bias;
+    fill_bias(&bias, sink_len, sink_bias, window, window_bias, kb_bias, kb_block,
+              kb_bias ? L / (kb_block > 0 ? kb_block : 1) : 0);
+    const int total = n_units * B;
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#pragma omp parallel for schedule(dynamic, 4)
+#endif
+    for (int x = 0; x < total; ++x) {
+        const int t = x / B, a = x % B;
+        const int h = units[t] / nQB, I = units[t] % nQB;
+        const int64_t i = (int64_t)I * B + a;
+        double* row = out + ((int64_t)t * B + a) * L;
+        row_probs(Q + ((int64_t)h * L + i) * d, K + (int64_t)h * L * d, d, i + 1, sigma, &bias, h, i,
+                  row);
+        for (int64_t j = i + 1; j < L; ++j) row[j] = 0.0;
+    }
+    return 0;
+}
+
 /* ---------------------------------------------------------------------------------------------
  * Retrieval oracle, [MF] s3.3 + s5.4, evaluated on given kept sets (so selection and retrieval
  * can be checked separately):

@@ -375,3 +375,52 @@ def test_kept_mass_invariants(oracle_mod):
                 assert abs(km - r.kept_mass[h, I]) < 1e-12
                 assert km >= p - 1e-12 or len(S) == I + 1
                 assert km - r.mass[h, I, S].min() < p
+
+
+# ---------------------------------------------------------------------------------------------
+# s2.1: the row log-normaliser the oracle stores next to the masses is log sum_j exp(s_ij) over
+# the causal, biased logits.  Pinned to a closed form and to torch's float64 logsumexp over logits
+# formed with a numpy matmul and the mask of the bias rule (not the oracle's own loops).
+# ---------------------------------------------------------------------------------------------
+def test_row_lse_zero_query_closed_form(oracle_mod):
+    """Q = 0, no bias: every causal logit is 0, so the row normaliser is log(i + 1) exactly."""
+    H, L, d, B = 2, 128, 16, 32
+    Q = np.zeros((H, L, d), np.float32)
+    K = np.random.default_rng(5).standard_normal((H, L, d)).astype(np.float32)
+    r = oracle_mod.compress(Q, K, 1 / math.sqrt(d), 0.9, B, None)
+    want = np.log(np.arange(1, L + 1, dtype=np.float64))
+    assert np.max(np.abs(r.lse - want[None])) < 1e-13
+
+
+@pytest.mark.parametrize("n,kw", [(2, dict(L=256, H_s=3)), (4, dict(L=512, H_s=2, block=128)),
+                                  (3, dict(L=256, H_s=2))])
+def test_row_lse_matches_torch_logsumexp(oracle_mod, n, kw):
+    """Biased causal logits (sink, window and key-block terms, max rule) -> torch.logsumexp."""
+    spec = _small(n, **kw)
+    lay = draw_layers(spec)[0]
+    r = oracle_mod.compress(lay.Q, lay.K, spec.scale, spec.p, spec.block, lay.bias)
+    Q = lay.Q.astype(np.float64)
+    K = lay.K.astype(np.float64)
+    logits = spec.scale * np.einsum("hid,hjd->hij", Q, K) + _mask_from_rule(spec.H_s, spec.L, spec.L, lay.bias)
+    want = torch.logsumexp(torch.from_numpy(logits), dim=-1).numpy()
+    assert np.max(np.abs(r.lse - want)) < 1e-11
+
+
+@pytest.mark.parametrize("n,kw", [(2, dict(L=256, H_s=3)), (4, dict(L=512, H_s=2, block=128))])
+def test_row_block_probs_match_torch_softmax(oracle_mod, n, kw):
+    """Whole query blocks of the map (s2.1) against torch's float64 softmax over the biased causal
+    logits (numpy matmul + the bias-rule mask), and against the single-tile oracle entry."""
+    spec = _small(n, **kw)
+    lay = draw_layers(spec)[0]
+    B, nqb = spec.block, spec.L // spec.block
+    units = [0, nqb - 1, (spec.H_s - 1) * nqb + nqb // 2]
+    got = oracle_mod.row_block_probs(lay.Q, lay.K, spec.scale, B, units, lay.bias)
+    logits = spec.scale * np.einsum("hid,hjd->hij", lay.Q.astype(np.float64), lay.K.astype(np.float64))
+    logits = logits + _mask_from_rule(spec.H_s, spec.L, spec.L, lay.bias)
+    ref = torch.softmax(torch.from_numpy(logits), dim=-1).numpy()
+    for t, u in enumerate(units):
+        h, I = divmod(u, nqb)
+        assert np.max(np.abs(got[t] - ref[h, I * B:(I + 1) * B])) < 1e-13
+        J = I // 2
+        tile = oracle_mod.tile_probs(lay.Q, lay.K, spec.scale, B, h, I, J, lay.bias)
+        assert np.array_equal(got[t][:, J * B:(J + 1) * B], tile)
