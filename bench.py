@@ -30,7 +30,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from cross_model_attention_mr_b200.workloads import config, draw_batch, draw_layers, shrink  # noqa: E402
+from cross_model_attention_mr_b200.workloads import config, draw_batch, draw_layers, iter_layers, shrink  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "prefill tokens/s for compress+retrieve at L=32K; % TC peak and % HBM peak"
@@ -114,13 +114,26 @@ def gpu_index_for(local_rank: int) -> str:
 # ------------------------------------------------------------------------------------------------
 # algorithmic work of the path (what the method must do, independent of the implementation)
 # ------------------------------------------------------------------------------------------------
-def algorithmic(spec, nnz: int, union_tiles: int, n_req: int = 1):
+def dense_causal_flops(H: int, d: int, d_v: int, first_pos: int, n_rows: int) -> int:
+    """QK^T and PV flops of exact causal attention for rows at positions first_pos .. + n_rows - 1
+    (row at position i sees i + 1 keys)."""
+    keys = n_rows * first_pos + n_rows * (n_rows + 1) // 2
+    return 2 * H * keys * (d + d_v)
+
+
+def algorithmic(spec, nnz: int, union_tiles: int, n_req: int = 1, suffixes=None, fp8: bool = False):
     B, d, L = spec.block, spec.d, spec.L
+    # bytes per stored tile: values (bf16, or e4m3 plus one fp32 scale per 32 x 64 piece) + column index
+    tile_bytes = (B * B + 4 * (B // 32) * (B // 64) if fp8 else B * B * 2) + 4
+    dense = 0
+    if suffixes is not None:  # receiver heads' dense rows after the shared prefix
+        dense = sum(dense_causal_flops(spec.H_r, d, spec.d_v, L, int(x)) for x in suffixes)
     return {
+        "dense_flops": dense,
         # one causal QK^T per sender head: H_s * d * L * (L + 1) flops
         "compress_flops": spec.H_s * d * L * (L + 1),
-        # the stored map: kept tiles of B*B bf16 probabilities plus one int32 column index each
-        "map_bytes": nnz * (B * B * 2 + 4),
+        # the stored map: kept tiles of B*B probabilities plus one int32 column index each
+        "map_bytes": nnz * tile_bytes,
         # translated map times V over the union of kept key blocks, per receiver head and request
         "retrieve_av_flops": spec.H_r * n_req * union_tiles * 2 * B * B * spec.d_v,
         # head mixing: each kept sender tile is weighted into every receiver head
@@ -129,16 +142,61 @@ def algorithmic(spec, nnz: int, union_tiles: int, n_req: int = 1):
 
 
 def kernel_work(name: str, work: dict):
-    """(bound, amount, unit) of a kernel's algorithmic work per launch."""
+    """(bound, amount, unit) of a kernel's algorithmic work per launch, against the roof the method
+    names for its stage: the tensor-core peak for the contractions (QK^T in compression; the head
+    mixing and X.V in retrieval), the HBM peak for writing the map."""
     if name in ("mr_compress_stats", "mr_compress_tc"):
         return "tensor", work["compress_flops"], "flop"
     if name in ("mr_emit", "mr_emit_tc"):
         return "hbm", work["map_bytes"], "byte"
     if name in ("mr_retrieve", "mr_retrieve_tc"):
-        # the binding arithmetic is the fp32 head mixing on the CUDA cores (FFMA); the X.V product
-        # on the tensor cores is a small fraction of its time
-        return "alu", work["retrieve_mix_flops"], "flop"
+        return "tensor", work["retrieve_av_flops"] + work["retrieve_mix_flops"], "flop"
+    if name in ("mr_dense", "mr_dense_tc"):
+        return "tensor", work.get("dense_flops", 0), "flop"
     return None, 0, None
+
+
+def stage_rooflines(prof: dict, work: dict, pk: dict, sms: int):
+    """Per launched kernel: algorithmic work / average launch time against the measured peaks
+    (tensor: bf16 sustained; hbm: copy bandwidth).  The retrieval also reports its map bytes
+    against HBM, and its fp32 head-mixing rate against the CUDA cores' FMA rate as a diagnostic
+    of the implementation (not the method's roof)."""
+    out = {}
+    tc_peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+    hbm_peak = float(pk["hbm_gbs"])
+    for name, (ms, cnt) in prof.items():
+        bound, amount, _ = kernel_work(name, work)
+        if bound is None or cnt == 0 or amount == 0:
+            continue
+        avg_s = ms / cnt / 1e3
+        e = {"ms_per_launch": ms / cnt, "bound": bound}
+        if bound == "tensor":
+            e.update(achieved_tflops=amount / avg_s / 1e12, peak_tflops=tc_peak,
+                     frac=amount / avg_s / 1e12 / tc_peak)
+        else:
+            e.update(achieved_gbs=amount / avg_s / 1e9, peak_gbs=hbm_peak, frac=amount / avg_s / 1e9 / hbm_peak)
+        if name in ("mr_retrieve", "mr_retrieve_tc"):
+            e["map_gbs"] = work["map_bytes"] / avg_s / 1e9
+            e["map_hbm_frac"] = e["map_gbs"] / hbm_peak
+            fma_peak = sms * 128 * 2 * float(pk.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+            e["diagnostic_fp32_mixing"] = {"achieved_tflops": work["retrieve_mix_flops"] / avg_s / 1e12,
+                                           "fp32_fma_peak_tflops": fma_peak,
+                                           "note": "head mixing on CUDA cores; the roof of that choice"}
+        out[name] = e
+    return out
+
+
+def roofline_of(name: str, ms: float, cnt: int, work: dict, pk: dict, pk_src: str):
+    """The bench line's roofline object for one kernel (its stage's roof, see kernel_work)."""
+    bound, amount, _ = kernel_work(name, work)
+    avg_s = ms / cnt / 1e3
+    if bound == "hbm":
+        achieved, peak, runit, kind = amount / avg_s / 1e9, float(pk["hbm_gbs"]), "GB/s", "copy"
+    else:
+        achieved, runit, kind = amount / avg_s / 1e12, "TFLOP/s", "bf16 sustained"
+        peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": runit, "frac": achieved / peak,
+            "traffic": None, "kernel": name, "peak_source": pk_src, "peak_kind": kind}
 
 
 def source_hash(files):
@@ -255,6 +313,15 @@ def job_tokens_per_s(world: int, L: int, ms: float) -> float:
     return world * L / (ms / 1e3)
 
 
+def line_config(spec, world: int) -> dict:
+    """The `config` of the headline line; the reference arm prints the same dict."""
+    return {"workload": spec.name, "L": spec.L, "H_s": spec.H_s, "H_r": spec.H_r, "d": spec.d,
+            "d_v": spec.d_v, "block": spec.block, "p": spec.p, "layers": 1,
+            "l2": "inputs larger than L2 (Q, K %d MB each, V %d MB, the map tens of GB)" % (
+                spec.H_s * spec.L * spec.d * 2 // 10**6, spec.H_r * spec.L * spec.d_v * 2 // 10**6),
+            "parallelism": f"replicas{world}"}
+
+
 def run_reference(args, spec, rank):
     if rank != 0:
         return
@@ -262,22 +329,25 @@ def run_reference(args, spec, rank):
     threads = os.cpu_count() or 1
     nqb = spec.L // spec.block
     rng = np.random.default_rng(11)
-    vals = []
+    vals, took = [], []
     desc = ""
     for step in range(args.warmup + args.steps):
         if step < args.warmup:  # warm-up: one small pass (page-in, thread pool start)
             u, r = rng.integers(nqb // 2, nqb, size=threads).tolist(), rng.integers(spec.L // 2, spec.L, size=threads).tolist()
             oracle_sample_time(spec, lay, u, r, threads)
             continue
+        t0 = time.perf_counter()
         t_full, desc = oracle_sample_calibrated(spec, lay, threads, 8.0, rng)
+        took.append(time.perf_counter() - t0)
         vals.append(spec.L / t_full)
     value = float(statistics.median(vals))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * spec.L / value,
+        "ms_per_step_extrapolated": True,
+        "sample_seconds_per_step": float(statistics.median(took)),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": spec.name, "L": spec.L, "H_s": spec.H_s, "H_r": spec.H_r,
-                                        "d": spec.d, "block": spec.block, "p": spec.p},
+        "data": "synthetic", "config": line_config(spec, args.gpus),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": "per step: " + desc},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -319,9 +389,9 @@ def run_config_line(args, spec, n):
     suffixes = None
     nqb = spec.L // spec.block
     if n in (2, 3):
-        layers = draw_layers(spec)
+        # layer by layer: each layer goes to the device before the next is drawn
         dev = [(to_dev(l.Q), to_dev(l.K), to_dev(l.V), torch.from_numpy(l.W).cuda(), mr.Bias.from_spec(l.bias))
-               for l in layers]
+               for l in iter_layers(spec)]
         ws_r = mr.Workspace(mr.retrieve_workspace_bytes(m, spec.H_r, spec.d_v, 1))
         O = torch.empty((1, spec.H_r, spec.L, spec.d_v), dtype=bf, device="cuda")
         wss = [ws_c, ws_r]
@@ -397,27 +467,17 @@ def run_config_line(args, spec, n):
     ms = ev0.elapsed_time(ev1) / args.steps
     tokens = config_tokens_per_step(spec, suffixes)
     n_req = spec.n_req if n == 5 else 1
-    per_layer = [algorithmic(spec, nnz, un, n_req) for nnz, un in maps]
+    per_layer = [algorithmic(spec, nnz, un, n_req, suffixes) for nnz, un in maps]
     work = {k: sum(w[k] for w in per_layer) / len(per_layer) for k in per_layer[0]}  # per launch, layer mean
     pk, pk_src = peaks()
     dname, (dms, dcnt) = max(prof.items(), key=lambda kv: kv[1][0])
-    bound, amount, _ = kernel_work(dname, work)
-    roofline = None
-    if bound is not None:
-        avg_s = dms / dcnt / 1e3
-        if bound == "hbm":
-            achieved, peak, runit, kind = amount / avg_s / 1e9, float(pk["hbm_gbs"]), "GB/s", "copy"
-        elif bound == "alu":
-            sms = torch.cuda.get_device_properties(0).multi_processor_count
-            achieved, runit, kind = amount / avg_s / 1e12, "TFLOP/s", "fp32 FMA"
-            peak, pk_src = sms * 128 * 2 * float(pk.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12, "derived"
-        else:
-            achieved, runit, kind = amount / avg_s / 1e12, "TFLOP/s", "sustained"
-            peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
-        roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": runit, "frac": achieved / peak,
-                    "traffic": None, "kernel": dname, "peak_source": pk_src, "peak_kind": kind}
+    roofline = roofline_of(dname, dms, dcnt, work, pk, pk_src)
+    roofline["traffic"] = None
     total = sum(v[0] for v in prof.values())
     stages = {k: {"ms_per_launch": v[0] / v[1], "launches": v[1], "share": v[0] / total} for k, v in prof.items()}
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for k, r in stage_rooflines(prof, work, pk, sms).items():
+        stages[k].update(r)
     nnz_all = sum(x[0] for x in maps)
     tiles_all = len(maps) * spec.H_s * nqb * (nqb + 1) / 2
     line = {
@@ -438,6 +498,121 @@ def run_config_line(args, spec, n):
 
 
 # ------------------------------------------------------------------------------------------------
+# the retrieval's map reads alone (gather-only measurement)
+# ------------------------------------------------------------------------------------------------
+def run_gather_probe(args, spec):
+    """Compress the workload once, then time mr_gather_probe: every stored tile moved to shared
+    memory by 1 CTA (from DRAM) and by 16 CTAs side by side (the retrieval's re-read factor at 4
+    receiver heads per CTA), with the retrieval's copy mechanism and no arithmetic."""
+    import torch
+    from cross_model_attention_mr_b200 import mr
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    lay = draw_layers(spec)[0]
+    bf = torch.bfloat16
+    fp8 = args.map == "fp8"
+    m = mr.compress(torch.from_numpy(lay.Q).to(bf).cuda(), torch.from_numpy(lay.K).to(bf).cuda(),
+                    float(np.float32(spec.p)), spec.block, bias=mr.Bias.from_spec(lay.bias), scale=spec.scale,
+                    map_dtype=mr.MR_FP8_E4M3 if fp8 else None)
+    torch.cuda.synchronize()
+    nnz = m.nnz_host()
+    tile_bytes = spec.block * spec.block * (1 if fp8 else 2)
+    pk, pk_src = peaks()
+    ws = mr.Workspace(256)
+    out = {}
+    for readers in (1, 16):
+        for _ in range(args.warmup):
+            mr.gather_probe(m, readers, ws, stream)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            mr.gather_probe(m, readers, ws, stream)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        ms = ev0.elapsed_time(ev1) / args.steps
+        gbs = readers * nnz * tile_bytes / (ms / 1e3) / 1e9
+        out[str(readers)] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / float(pk["hbm_gbs"])}
+    line = {"metric": "map gather alone: stored tiles moved to shared memory, GB/s", "unit": "GB/s",
+            "value": out["1"]["GB/s"], "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "dtype": "fp8" if fp8 else "bf16", "data": "synthetic",
+            "config": {"workload": spec.name, "map_tiles": nnz, "tile_bytes": tile_bytes,
+                       "map_bytes": nnz * tile_bytes},
+            "readers": out, "peak_gbs": float(pk["hbm_gbs"]), "peak_source": pk_src}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------------
+# one sequence split across ranks (strong scaling)
+# ------------------------------------------------------------------------------------------------
+def run_split(args, spec, dist, world: int, rank: int, local: int):
+    """Each rank owns a contiguous, work-balanced range of query blocks and the token rows of that
+    range.  A step all-gathers the ranks' K and V row shards (the path's one exchange), then
+    compresses its query blocks and retrieves its output rows; maps and outputs stay local.
+    value = L / (slowest rank's step time)."""
+    import torch
+    from cross_model_attention_mr_b200 import mr
+    torch.cuda.set_device(local)
+    stream = torch.cuda.current_stream()
+    bf = torch.bfloat16
+    lay = draw_layers(spec)[0]
+    nqb = spec.L // spec.block
+    ranges = mr.split_query_blocks(nqb, world, 1 if spec.block == 128 else 2)
+    shards = mr.row_shards(spec.L, ranges, spec.block)
+    q0, q1 = ranges[rank]
+    b, e = shards[rank]
+    Q = torch.from_numpy(lay.Q).to(bf).cuda()   # rows outside this rank's range are never read
+    Kl = torch.from_numpy(np.ascontiguousarray(lay.K[:, b:e])).to(bf).cuda()
+    Vl = torch.from_numpy(np.ascontiguousarray(lay.V[:, b:e])).to(bf).cuda()
+    W = torch.from_numpy(lay.W).cuda()
+    bias = mr.Bias.from_spec(lay.bias)
+    p = float(np.float32(spec.p))
+    m = mr.Map(spec.H_s, spec.L, spec.block, mr.MR_BF16, max(1, mr.max_tiles(spec.H_s, spec.L, spec.block)), "cuda")
+    ws_c = mr.Workspace(mr.compress_workspace_bytes(spec.H_s, spec.L, spec.d, spec.block))
+    ws_r = mr.Workspace(mr.retrieve_workspace_bytes(m, spec.H_r, spec.d_v, 1))
+    O = torch.empty((1, spec.H_r, spec.L, spec.d_v), dtype=bf, device="cuda")
+
+    def step():
+        K = mr.gather_row_shards(Kl, shards) if world > 1 else Kl
+        V = mr.gather_row_shards(Vl, shards) if world > 1 else Vl
+        if q1 > q0:
+            mr.compress(Q, K, p, spec.block, bias=bias, scale=spec.scale, out=m, ws=ws_c, stream=stream,
+                        blocks=(q0, q1))
+            mr.retrieve(m, W, V, out=O, ws=ws_r, stream=stream, blocks=(q0, q1))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ok = (q1 == q0) or not (ws_c.sync_status() or ws_r.sync_status())
+    if not all_ranks_ok(ok, dist, "cuda"):
+        raise SystemExit("device status after warm-up")
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dist, "cuda")
+    ok = (q1 == q0) or not (ws_c.sync_status() or ws_r.sync_status())
+    if not all_ranks_ok(ok, dist, "cuda"):
+        raise SystemExit("device status in the timed steps")
+    if rank == 0:
+        line = {
+            "metric": METRIC + " (one sequence split across ranks)", "value": spec.L / (ms / 1e3),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(line_config(spec, world), parallelism=f"query-block split x{world}",
+                           ranges=[list(r) for r in ranges]),
+            "exchange": "all-gather of K and V row shards per step (torch.distributed)",
+        }
+        print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------------
 # native arm
 # ------------------------------------------------------------------------------------------------
 def main():
@@ -451,6 +626,12 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--L", type=int, default=None,
                     help="shorter sequence of the same workload shape (profiling captures); default 32768")
+    ap.add_argument("--gather-probe", action="store_true",
+                    help="time the retrieval's map reads alone (mr_gather_probe) on the workload's map")
+    ap.add_argument("--split", action="store_true",
+                    help="split one sequence across the ranks by query-block range (strong scaling)")
+    ap.add_argument("--map", default="bf16", choices=["bf16", "fp8"],
+                    help="map value type: bf16 (default, the headline) or fp8 (e4m3 with per-piece scales)")
     ap.add_argument("--config", type=int, default=4, choices=[2, 3, 4, 5],
                     help="workload: 4 = the headline line (default); 2, 3, 5 = one-GPU measurement lines")
     args = ap.parse_args()
@@ -463,6 +644,9 @@ def main():
     if args.L is not None and args.L != spec.L:
         name = spec.name.replace("L32768", f"L{args.L}") if "L32768" in spec.name else f"{spec.name}_at_L{args.L}"
         spec = shrink(spec, L=args.L, name=name)
+    if args.gather_probe:
+        run_gather_probe(args, spec)
+        return
     if args.config != 4 and args.impl != "reference":
         if int(os.environ.get("WORLD_SIZE", "1")) > 1:
             raise SystemExit("--config 2/3/5 lines are one-GPU measurements")
@@ -483,6 +667,13 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
+    if args.split:
+        try:
+            run_split(args, spec, dist, world, rank, local)
+        finally:
+            if dist is not None:
+                dist.destroy_process_group()
+        return
     spec = rank_spec(spec, rank)  # independent sequence per rank
 
     lay = draw_layers(spec)[0]
@@ -497,7 +688,8 @@ def main():
     bias = mr.Bias.from_spec(lay.bias)
     p = float(np.float32(spec.p))
     cap = mr.max_tiles(spec.H_s, spec.L, spec.block)
-    m = mr.Map(spec.H_s, spec.L, spec.block, mr.MR_BF16, cap, "cuda")
+    fp8 = args.map == "fp8"
+    m = mr.Map(spec.H_s, spec.L, spec.block, mr.MR_FP8_E4M3 if fp8 else mr.MR_BF16, cap, "cuda")
     ws_c = mr.Workspace(mr.compress_workspace_bytes(spec.H_s, spec.L, spec.d, spec.block))
     ws_r = mr.Workspace(mr.retrieve_workspace_bytes(m, spec.H_r, spec.d_v, 1))
     O = torch.empty((1, spec.H_r, spec.L, spec.d_v), dtype=bf, device="cuda")
@@ -521,7 +713,7 @@ def main():
     kept = m.kept_bits_host()
     nqb = spec.L // spec.block
     union_tiles = int(np.any(kept, axis=0).sum())
-    work = algorithmic(spec, nnz, union_tiles)
+    work = algorithmic(spec, nnz, union_tiles, fp8=fp8)
 
     # ---- timed region (device time, CUDA events on the launching stream) ----
     sampler = ClockSampler(gpu_index_for(local))
@@ -549,30 +741,16 @@ def main():
     ms = max_over_ranks(ms, dist, "cuda")
     value = job_tokens_per_s(world, spec.L, ms)
 
-    # ---- roofline of the dominant kernel ----
+    # ---- roofline of the dominant kernel, and of every stage ----
     pk, pk_src = peaks()
-    dom = max(prof.items(), key=lambda kv: kv[1][0])
-    dname, (dms, dcnt) = dom
-    bound, amount, unit = kernel_work(dname, work)
-    avg_s = dms / dcnt / 1e3
-    peak_kind = "sustained"
-    if bound == "hbm":
-        achieved, peak, runit = amount / avg_s / 1e9, float(pk["hbm_gbs"]), "GB/s"
-        peak_kind = "copy"
-    elif bound == "alu":
-        # fp32 FMA peak from unit counts and the clock: SMs x 128 FMA lanes x 2 flop x max SM clock
-        sms = torch.cuda.get_device_properties(local).multi_processor_count
-        mhz = float(pk.get("sm_max_mhz", 1965.0))
-        achieved = amount / avg_s / 1e12
-        peak, runit, pk_src, peak_kind = sms * 128 * 2 * mhz * 1e6 / 1e12, "TFLOP/s", "derived", "fp32 FMA"
-    else:
-        achieved = amount / avg_s / 1e12
-        peak, runit = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])), "TFLOP/s"
-    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": runit, "frac": achieved / peak,
-                "traffic": traffic_for(dname), "kernel": dname, "peak_source": pk_src,
-                "peak_kind": peak_kind}
+    dname, (dms, dcnt) = max(prof.items(), key=lambda kv: kv[1][0])
+    roofline = roofline_of(dname, dms, dcnt, work, pk, pk_src)
+    roofline["traffic"] = traffic_for(dname)
     stages = {k: {"ms_per_launch": v[0] / v[1], "launches": v[1], "share": v[0] / sum(x[0] for x in prof.values())}
               for k, v in prof.items()}
+    sms = torch.cuda.get_device_properties(local).multi_processor_count
+    for k, r in stage_rooflines(prof, work, pk, sms).items():
+        stages[k].update(r)
 
     # ---- end to end through the public API with host buffers ----
     # Every step copies its inputs from pinned host memory and reads its result back inside the
@@ -646,8 +824,12 @@ def main():
         d1.record(stream)
         _t.cuda.synchronize()
         dms_ = d0.elapsed_time(d1)
-        dense = {"tokens_per_s": spec.L / (dms_ / 1e3), "ms": dms_, "heads": spec.H_r,
-                 "flops": 2 * spec.H_r * spec.L * (spec.L + 1) * (spec.d + spec.d_v) // 2}
+        dfl = dense_causal_flops(spec.H_r, spec.d, spec.d_v, 0, spec.L)
+        pkd, _ = peaks()
+        dense = {"tokens_per_s": spec.L / (dms_ / 1e3), "ms": dms_, "heads": spec.H_r, "flops": dfl,
+                 "achieved_tflops": dfl / (dms_ / 1e3) / 1e12,
+                 "frac_of_bf16_burst": dfl / (dms_ / 1e3) / 1e12 / float(pkd["bf16_tflops"]),
+                 "note": "exact causal attention of the receiver heads, one launch timed alone"}
         del Qr, Kr, Od
 
     # ---- CPU oracle baseline (rank 0, N = 1 only) ----
@@ -662,12 +844,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Gaussian Q/K/V, sink+window+retrieval-block logit bias, row-softmax W)",
-            "config": {"workload": spec.name, "L": spec.L, "H_s": spec.H_s, "H_r": spec.H_r, "d": spec.d,
-                       "d_v": spec.d_v, "block": spec.block, "p": spec.p, "layers": 1,
-                       "l2": "inputs larger than L2 (Q,K %d MB each, V %d MB, map %.1f GB)" % (
-                           spec.H_s * spec.L * spec.d * 2 // 10**6, spec.H_r * spec.L * spec.d_v * 2 // 10**6,
-                           work["map_bytes"] / 1e9),
-                       "parallelism": f"replicas{world}"},
+            "config": dict(line_config(spec, world), **({"map_values": "fp8 e4m3, scale per 32 x 64 piece"} if fp8 else {})),
             "gpu_launches": int(launches),
             "clocks": clocks,
             "roofline": roofline,

@@ -91,9 +91,9 @@ int64_t mr_bsr_max_tiles(int H_s, int L, int block) {
   return (int64_t)H_s * nqb * (nqb + 1) / 2;
 }
 
-mr_status mr_compress(const void* Q, const void* K, mr_dtype dt, int H_s, int L, int d, float scale,
-                      float p, const mr_logit_bias* bias, mr_bsr* out, void* ws, size_t ws_bytes,
-                      void* stream) {
+mr_status mr_compress_blocks(const void* Q, const void* K, mr_dtype dt, int H_s, int L, int d,
+                             float scale, float p, const mr_logit_bias* bias, int qb_begin,
+                             int qb_end, mr_bsr* out, void* ws, size_t ws_bytes, void* stream) {
   if (!Q || !K || !out || !ws) return MR_ERR_INVALID_ARG;
   if (dt != MR_BF16 && dt != MR_F32) return MR_ERR_INVALID_ARG;
   if (!isfinite(scale) || !(p > 0.f) || isnan(p)) return MR_ERR_INVALID_ARG;
@@ -101,11 +101,16 @@ mr_status mr_compress(const void* Q, const void* K, mr_dtype dt, int H_s, int L,
   if (out->block < 1 || L % out->block) return MR_ERR_UNSUPPORTED;
   if (!shape_ok(H_s, L, d, out->block)) return MR_ERR_UNSUPPORTED;
   if (out->H_s != H_s || out->L != L) return MR_ERR_INVALID_ARG;
-  if (out->val_dtype != dt) return MR_ERR_UNSUPPORTED;
+  const bool fp8 = out->val_dtype == MR_FP8_E4M3;
+  if (out->val_dtype != dt && !(fp8 && dt == MR_BF16)) return MR_ERR_UNSUPPORTED;
+  if (fp8 && d != 128) return MR_ERR_UNSUPPORTED;  // fp8 maps come from the tensor-core emit only
+  if (fp8 && out->capacity_tiles > 0 && !out->tile_scale) return MR_ERR_INVALID_ARG;
   if (out->capacity_tiles < 0) return MR_ERR_INVALID_ARG;
   if (!out->row_ptr || !out->kept_mass || !out->kept_bits || !out->nnz) return MR_ERR_INVALID_ARG;
   if (out->capacity_tiles > 0 && (!out->col_idx || !out->vals)) return MR_ERR_INVALID_ARG;
   if (mr_bsr_max_tiles(H_s, L, out->block) >= ((int64_t)1 << 31)) return MR_ERR_UNSUPPORTED;
+  const int nqb = L / out->block;
+  if (qb_begin < 0 || qb_end > nqb || qb_begin >= qb_end) return MR_ERR_INVALID_ARG;
   const mr_status bs = bias_ok(bias, L);
   if (bs != MR_OK) return bs;
   const CompressLayout lay = compress_layout(H_s, L, out->block);
@@ -128,12 +133,31 @@ mr_status mr_compress(const void* Q, const void* K, mr_dtype dt, int H_s, int L,
   a.ws = (WsHeader*)ws;
   a.lse_ws = (float*)((char*)ws + lay.lse_off);
   a.count_ws = (int*)((char*)ws + lay.count_off);
+  a.qb0 = qb_begin;
+  a.qb1 = qb_end;
   a.map = *out;
   a.stream = st;
-  if (!tc_compress_supported(a)) return from_cuda(simt_compress(a));
+  if (qb_begin > 0 || qb_end < nqb) {
+    // rows outside the range are empty: zero counts, kept bits, kept masses (and stored masses)
+    const size_t rows = (size_t)H_s * nqb, words = (size_t)(nqb + 31) / 32;
+    if (cudaMemsetAsync(a.count_ws, 0, rows * sizeof(int), st) != cudaSuccess ||
+        cudaMemsetAsync(out->kept_bits, 0, rows * words * sizeof(uint32_t), st) != cudaSuccess ||
+        cudaMemsetAsync(out->kept_mass, 0, rows * sizeof(float), st) != cudaSuccess ||
+        (out->mass && cudaMemsetAsync(out->mass, 0, rows * nqb * sizeof(float), st) != cudaSuccess))
+      return MR_ERR_CUDA;
+  }
+  if (!tc_compress_supported(a)) return fp8 ? MR_ERR_UNSUPPORTED : from_cuda(simt_compress(a));
   if ((e = tc_compress_stats(a)) != cudaSuccess) return MR_ERR_CUDA;
-  if ((e = launch_scan_counts(a.count_ws, H_s * (L / out->block), a.map, a.ws, st)) != cudaSuccess) return MR_ERR_CUDA;
+  if ((e = launch_scan_counts(a.count_ws, H_s * nqb, a.map, a.ws, st)) != cudaSuccess) return MR_ERR_CUDA;
   return from_cuda(tc_emit(a));
+}
+
+mr_status mr_compress(const void* Q, const void* K, mr_dtype dt, int H_s, int L, int d, float scale,
+                      float p, const mr_logit_bias* bias, mr_bsr* out, void* ws, size_t ws_bytes,
+                      void* stream) {
+  if (!out) return MR_ERR_INVALID_ARG;
+  if (out->block < 1 || L < 1 || L % out->block) return L < 1 ? MR_ERR_INVALID_ARG : MR_ERR_UNSUPPORTED;
+  return mr_compress_blocks(Q, K, dt, H_s, L, d, scale, p, bias, 0, L / out->block, out, ws, ws_bytes, stream);
 }
 
 size_t mr_retrieve_workspace_bytes(const mr_bsr* map, int H_r, int d_v, int n_req) {
@@ -144,19 +168,42 @@ size_t mr_retrieve_workspace_bytes(const mr_bsr* map, int H_r, int d_v, int n_re
   return kRetrieveWsBytes;
 }
 
-mr_status mr_retrieve(const mr_bsr* map, const float* W, int H_r, const void* V, void* O,
-                      mr_dtype dt, int d_v, int n_req, const int64_t* v_req_off,
-                      int64_t v_req_stride, int64_t v_head_stride, void* ws, size_t ws_bytes,
-                      void* stream) {
+mr_status mr_retrieve(const mr_bsr* map, const float* W, int H_r, const void* V, int64_t v_elems,
+                      void* O, mr_dtype dt, int d_v, int n_req, const int64_t* v_req_off,
+                      int64_t v_req_stride, int64_t v_head_stride, const mr_retrieve_opts* opts,
+                      void* ws, size_t ws_bytes, void* stream) {
   if (!map || !W || !V || !O || !ws) return MR_ERR_INVALID_ARG;
   if (dt != MR_BF16 && dt != MR_F32) return MR_ERR_INVALID_ARG;
-  if (H_r < 1 || n_req < 1 || v_head_stride < 0 || v_req_stride < 0) return MR_ERR_INVALID_ARG;
+  if (H_r < 1 || n_req < 1 || v_head_stride < 0 || v_req_stride < 0 || v_elems < 1) return MR_ERR_INVALID_ARG;
   if (H_r > 256) return MR_ERR_UNSUPPORTED;
   if (d_v != 64 && d_v != 128) return MR_ERR_UNSUPPORTED;
   if (!shape_ok(map->H_s, map->L, 64, map->block)) return MR_ERR_UNSUPPORTED;
-  if (map->val_dtype != dt) return MR_ERR_UNSUPPORTED;
+  const bool fp8 = map->val_dtype == MR_FP8_E4M3;
+  if (map->val_dtype != dt && !(fp8 && dt == MR_BF16)) return MR_ERR_UNSUPPORTED;
   if (!map->row_ptr || !map->kept_bits || !map->vals) return MR_ERR_INVALID_ARG;
-  if (v_head_stride < (int64_t)map->L * d_v) return MR_ERR_INVALID_ARG;
+  if (fp8 && !map->tile_scale) return MR_ERR_INVALID_ARG;
+  const int nqb = map->L / map->block;
+  int qb0 = 0, qb1 = nqb, group = 1;
+  if (opts) {
+    if (opts->qb_begin != 0 || opts->qb_end != 0) {
+      qb0 = opts->qb_begin;
+      qb1 = opts->qb_end;
+      if (qb0 < 0 || qb1 > nqb || qb0 >= qb1) return MR_ERR_INVALID_ARG;
+    }
+    if (opts->v_group < 0) return MR_ERR_INVALID_ARG;
+    group = opts->v_group > 1 ? opts->v_group : 1;
+    if (H_r % group) return MR_ERR_INVALID_ARG;
+  }
+  const int H_v = H_r / group;
+  const int64_t seq = (int64_t)map->L * d_v;
+  if (H_v > 1 && v_head_stride < seq) return MR_ERR_INVALID_ARG;
+  // strided values: the furthest element read must lie inside the allocation
+  if (!v_req_off) {
+    const int64_t last = (int64_t)(n_req - 1) * v_req_stride + (int64_t)(H_v - 1) * v_head_stride + seq;
+    if (last > v_elems) return MR_ERR_INVALID_ARG;
+  } else if (seq > v_elems) {
+    return MR_ERR_INVALID_ARG;
+  }
   if (ws_bytes < mr_retrieve_workspace_bytes(map, H_r, d_v, n_req)) return MR_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
   if (cudaMemsetAsync(ws, 0, kRetrieveWsBytes, st) != cudaSuccess) return MR_ERR_CUDA;  // header + progress
@@ -165,6 +212,7 @@ mr_status mr_retrieve(const mr_bsr* map, const float* W, int H_r, const void* V,
   a.W = W;
   a.H_r = H_r;
   a.V = V;
+  a.v_elems = v_elems;
   a.O = O;
   a.dt = dt;
   a.d_v = d_v;
@@ -172,6 +220,9 @@ mr_status mr_retrieve(const mr_bsr* map, const float* W, int H_r, const void* V,
   a.v_req_off = v_req_off;
   a.v_req_stride = v_req_stride;
   a.v_head_stride = v_head_stride;
+  a.v_group = group;
+  a.qb0 = qb0;
+  a.qb1 = qb1;
   a.ws = (WsHeader*)ws;
   a.stream = st;
   return from_cuda(tc_retrieve_supported(a) ? tc_retrieve(a) : simt_retrieve(a));
@@ -215,7 +266,7 @@ mr_status mr_dense_ref(const void* Q, const void* K, const void* V, void* O, mr_
   a.bias = make_bias(bias);
   a.ws = (WsHeader*)ws;
   a.stream = st;
-  return from_cuda(simt_dense(a));
+  return from_cuda(tc_dense_supported(a) ? tc_dense(a) : simt_dense(a));
 }
 
 mr_status mr_sync_status(void* ws, void* stream) {
@@ -237,8 +288,18 @@ mr_status mr_bsr_nnz(const mr_bsr* map, int64_t* nnz_host, void* stream) {
 
 mr_status mr_bsr_export(const mr_bsr* map, int64_t n_tiles, float* out, void* stream) {
   if (!map || !out || n_tiles < 0 || (n_tiles > 0 && !map->vals)) return MR_ERR_INVALID_ARG;
+  if (map->val_dtype == MR_FP8_E4M3 && n_tiles > 0 && !map->tile_scale) return MR_ERR_INVALID_ARG;
   if (n_tiles > map->capacity_tiles) return MR_ERR_INVALID_ARG;
   return from_cuda(launch_export(*map, n_tiles, out, (cudaStream_t)stream));
+}
+
+mr_status mr_gather_probe(const mr_bsr* map, int readers, void* ws, size_t ws_bytes, void* stream) {
+  if (!map || !ws || readers < 1 || readers > 1024 || ws_bytes < kWsHeaderBytes) return MR_ERR_INVALID_ARG;
+  if (!shape_ok(map->H_s, map->L, 64, map->block)) return MR_ERR_UNSUPPORTED;
+  if (!map->row_ptr || !map->kept_bits || !map->vals) return MR_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (reset_header(ws, st) != cudaSuccess) return MR_ERR_CUDA;
+  return from_cuda(launch_gather_probe(*map, readers, (WsHeader*)ws, st));
 }
 
 }  // extern "C"

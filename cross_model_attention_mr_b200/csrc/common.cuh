@@ -109,6 +109,18 @@ __host__ __device__ __forceinline__ void tile_coords(int p, int B, int& a, int& 
   b = panel * P + ((pc ^ (a & 7)) * E) + (rem % E);
 }
 
+// Storage order of an fp8 (e4m3) tile: panels of 64 columns, rows of 64 bytes, no swizzle.
+__host__ __device__ __forceinline__ int tile_offset_fp8(int a, int b, int B) {
+  return (b >> 6) * B * 64 + a * 64 + (b & 63);
+}
+// Scales per fp8 tile (one per 32-row x 64-column piece) and the index of element (a, b)'s scale.
+__host__ __device__ __forceinline__ int fp8_scales_per_tile(int B) { return (B / 32) * (B / 64); }
+__host__ __device__ __forceinline__ int fp8_scale_index(int a, int b, int B) {
+  return (a >> 5) * (B / 64) + (b >> 6);
+}
+// Largest finite e4m3 value: a piece's values are stored as value / scale with scale = max / 448.
+constexpr float kFp8Max = 448.f;
+
 // Rank of key block J among the kept blocks of one row: number of kept blocks below J.
 __device__ __forceinline__ int kept_rank(const uint32_t* bits, int J) {
   int r = 0;

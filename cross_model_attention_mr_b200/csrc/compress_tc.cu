@@ -45,6 +45,8 @@ constexpr float kRescale = 8.0f;  // move the row reference only for a jump of m
 
 struct Params {
   int H, L, B, nqb, nkw, n_rb, n_units;
+  int rb_hi;     // units cover 128-row blocks rb_hi - n_rb .. rb_hi - 1
+  int qb0, qb1;  // query blocks whose selection is written
   float a;  // logit scale in base 2: scale * log2(e)
   float p;
   Bias bias;
@@ -83,7 +85,7 @@ __device__ __forceinline__ void fail(Smem& s, const Params& p, uint32_t detail) 
 }
 
 __device__ __forceinline__ void unit_of(const Params& p, int k, int& h, int& rb) {
-  rb = p.n_rb - 1 - k / p.H;
+  rb = p.rb_hi - 1 - k / p.H;
   h = k % p.H;
 }
 
@@ -376,7 +378,7 @@ __device__ void softmax_group(Smem& s, const Params& p, int w) {
 
     // ---- selection: warpgroup w selects query block w of the unit ----
     const int I = (p.B == 128) ? rb : 2 * rb + w;
-    const bool sel = (w < nblk) && I < p.nqb && good;
+    const bool sel = (w < nblk) && I < p.nqb && I >= p.qb0 && I < p.qb1 && good;
     const uint32_t bar_id = 2 + w;
     if (sel) {
       const int n = I + 1;
@@ -512,8 +514,13 @@ cudaError_t tc_compress_stats(const CompressArgs& a) {
   p.B = a.block;
   p.nqb = a.L / a.block;
   p.nkw = (p.nqb + 31) / 32;
-  p.n_rb = (a.L + 127) / 128;
+  // 128-row blocks holding the query blocks qb0 .. qb1 - 1
+  const int rb_lo = a.block == 128 ? a.qb0 : a.qb0 / 2;
+  p.rb_hi = a.block == 128 ? a.qb1 : (a.qb1 + 1) / 2;
+  p.n_rb = p.rb_hi - rb_lo;
   p.n_units = p.H * p.n_rb;
+  p.qb0 = a.qb0;
+  p.qb1 = a.qb1;
   p.a = a.scale * kLog2e;
   p.p = a.p;
   p.bias = a.bias;

@@ -12,6 +12,7 @@
 // tiles), MMA warp (128 x 128 tiles into two Tensor Memory buffers), two warpgroups that take
 // alternate needed tiles (one query row per thread).  All waits are bounded.
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -34,6 +35,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 struct Params {
   int H, L, B, nqb, nkw, n_rb, n_units;
+  int rb_hi;  // units cover 128-row blocks rb_hi - n_rb .. rb_hi - 1
   float a;
   Bias bias;
   const float* lse_ws;
@@ -41,7 +43,9 @@ struct Params {
   const uint32_t* kept_bits;
   int64_t capacity;
   int32_t* col_idx;
-  __nv_bfloat16* vals;
+  __nv_bfloat16* vals;   // bf16 maps
+  uint8_t* vals8;        // fp8 (e4m3) maps
+  float* tile_scale;     // fp8 maps: one scale per 32-row x 64-key piece
   WsHeader* ws;
 };
 
@@ -63,7 +67,7 @@ __device__ __forceinline__ void fail(Smem& s, const Params& p, uint32_t detail) 
 }
 
 __device__ __forceinline__ void unit_of(const Params& p, int k, int& h, int& rb) {
-  rb = p.n_rb - 1 - k / p.H;
+  rb = p.rb_hi - 1 - k / p.H;
   h = k % p.H;
 }
 
@@ -232,6 +236,7 @@ __device__ __forceinline__ float kb_offset(const Bias& b, int h, int j) {
 // One warpgroup: each warp handles 32 query rows of every tile given to the warpgroup, stages
 // them in the map's storage order and stores them with its own bulk copies (the 32 rows of a
 // panel are contiguous in the stored tile), so the warps of the group never wait on each other.
+template <bool F8>
 __device__ void emit_group(Smem& s, const Params& p, int w) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q4 = warp & 3;
@@ -275,6 +280,7 @@ __device__ void emit_group(Smem& s, const Params& p, int w) {
                            (p.bias.window > 0 && j_tile + 127 > 128 * rb - p.bias.window);
       // which 64-key halves of this warp's rows are stored
       const uint32_t row_mask = p.B == 128 ? 3u : ((pieces >> (2 * rh)) & 3u);
+      float sc[2] = {0.f, 0.f};  // fp8: scale of each stored piece
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t raw[2][32];
@@ -287,35 +293,58 @@ __device__ void emit_group(Smem& s, const Params& p, int w) {
           if (lane == 0) mbar_arrive(&s.s_empty[w]);
         }
         if (!((row_mask >> hh) & 1u)) continue;  // warp-uniform
-        char* dst = stage + 4096 * hh + lane * 128;
+        float pr[64];
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int j0 = j_tile + 64 * hh + 32 * cc;
-          float pr[32];
           if (!special) {
             const float o = kb_offset(p.bias, h, j0) - lse2;
 #pragma unroll
-            for (int t = 0; t < 32; ++t) pr[t] = ex2_approx(fmaf(__uint_as_float(raw[cc][t]), p.a, o));
+            for (int t = 0; t < 32; ++t) pr[32 * cc + t] = ex2_approx(fmaf(__uint_as_float(raw[cc][t]), p.a, o));
           } else {
             const float kb = kb_term(p.bias, h, j0);
 #pragma unroll
             for (int t = 0; t < 32; ++t) {
               const int j = j0 + t;
-              pr[t] = (row_ok && j <= i)
-                          ? ex2_approx(fmaf(__uint_as_float(raw[cc][t]), p.a, bias_with_kb(p.bias, i, j, kb) * kLog2e) - lse2)
-                          : 0.f;
+              pr[32 * cc + t] = (row_ok && j <= i)
+                                    ? ex2_approx(fmaf(__uint_as_float(raw[cc][t]), p.a, bias_with_kb(p.bias, i, j, kb) * kLog2e) - lse2)
+                                    : 0.f;
             }
           }
+        }
+        if (!F8) {
+          char* dst = stage + 4096 * hh + lane * 128;
 #pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
+          for (int c8 = 0; c8 < 8; ++c8) {  // 16-byte chunk of the 64-column panel row, swizzled
             uint32_t pk[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const __nv_bfloat162 b2 = __floats2bfloat162_rn(pr[8 * c8 + 2 * e], pr[8 * c8 + 2 * e + 1]);
               pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
             }
-            const int chunk = 4 * cc + c8;  // 16-byte chunk within the 64-column panel row
-            *reinterpret_cast<uint4*>(dst + ((chunk ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(dst + ((c8 ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        } else {
+          // the warp's 32 rows x 64 keys are one piece: scale = max / 448, values stored as e4m3
+          float mx = 0.f;
+#pragma unroll
+          for (int t = 0; t < 64; ++t) mx = fmaxf(mx, pr[t]);
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          sc[hh] = mx / kFp8Max;
+          const float inv = mx > 0.f ? kFp8Max / mx : 0.f;
+          char* dst = stage + 2048 * hh + lane * 64;
+#pragma unroll
+          for (int c16 = 0; c16 < 4; ++c16) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int x = 16 * c16 + 4 * e;
+              const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(pr[x] * inv, pr[x + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+              const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(pr[x + 2] * inv, pr[x + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+              pk[e] = lo | (hi << 16);
+            }
+            *reinterpret_cast<uint4*>(dst + 16 * c16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         }
       }
@@ -329,10 +358,19 @@ __device__ void emit_group(Smem& s, const Params& p, int w) {
           const int64_t t = tpos[piece];
           if (t >= p.capacity) continue;
           // destination: panel hh of the 128-tile, or the (rh, hh) 64-tile; this warp's 32 rows
-          const int64_t tbytes = (int64_t)p.B * p.B * 2;
-          char* gdst = reinterpret_cast<char*>(p.vals) + t * tbytes +
-                       (p.B == 128 ? 16384 * hh + 4096 * q4 : 4096 * (q4 & 1));
-          bulk_s2g(gdst, stage + 4096 * hh, 4096);
+          if (!F8) {
+            const int64_t tbytes = (int64_t)p.B * p.B * 2;
+            char* gdst = reinterpret_cast<char*>(p.vals) + t * tbytes +
+                         (p.B == 128 ? 16384 * hh + 4096 * q4 : 4096 * (q4 & 1));
+            bulk_s2g(gdst, stage + 4096 * hh, 4096);
+          } else {
+            const int64_t tbytes = (int64_t)p.B * p.B;
+            char* gdst = reinterpret_cast<char*>(p.vals8) + t * tbytes +
+                         (p.B == 128 ? 8192 * hh + 2048 * q4 : 2048 * (q4 & 1));
+            bulk_s2g(gdst, stage + 2048 * hh, 2048);
+            const int rg = p.B == 128 ? q4 : (q4 & 1);
+            p.tile_scale[t * fp8_scales_per_tile(p.B) + rg * (p.B / 64) + (p.B == 128 ? hh : 0)] = sc[hh];
+          }
           issued = true;
           const bool writer = p.B == 128 ? (q4 == 0 && hh == 0) : ((q4 & 1) == 0);
           if (writer) p.col_idx[t] = p.B == 128 ? T : 2 * T + hh;
@@ -349,6 +387,7 @@ __device__ void emit_group(Smem& s, const Params& p, int w) {
   __syncwarp();
 }
 
+template <bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     k_emit_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk, Params p) {
   extern __shared__ unsigned char smem_raw[];
@@ -381,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   else if (warp == kMmaWarp)
     mma_issuer(s, p);
   else if (warp >= kSoftmaxWarp0)
-    emit_group(s, p, (warp - kSoftmaxWarp0) >> 2);
+    emit_group<F8>(s, p, (warp - kSoftmaxWarp0) >> 2);
   __syncwarp();
   tc_fence_before();
   __syncthreads();
@@ -398,7 +437,10 @@ cudaError_t tc_emit(const CompressArgs& a) {
   p.B = a.block;
   p.nqb = a.L / a.block;
   p.nkw = (p.nqb + 31) / 32;
-  p.n_rb = (a.L + 127) / 128;
+  // rows of query blocks outside qb0 .. qb1 - 1 keep no tiles (their counts are 0)
+  const int rb_lo = a.block == 128 ? a.qb0 : a.qb0 / 2;
+  p.rb_hi = a.block == 128 ? a.qb1 : (a.qb1 + 1) / 2;
+  p.n_rb = p.rb_hi - rb_lo;
   p.n_units = p.H * p.n_rb;
   p.a = a.scale * kLog2e;
   p.bias = a.bias;
@@ -408,6 +450,8 @@ cudaError_t tc_emit(const CompressArgs& a) {
   p.capacity = a.map.capacity_tiles;
   p.col_idx = a.map.col_idx;
   p.vals = (__nv_bfloat16*)a.map.vals;
+  p.vals8 = (uint8_t*)a.map.vals;
+  p.tile_scale = a.map.tile_scale;
   p.ws = a.ws;
   CUtensorMap tq, tk;
   const uint64_t rows = (uint64_t)a.H * a.L;
@@ -418,10 +462,12 @@ cudaError_t tc_emit(const CompressArgs& a) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = p.n_units < sms ? p.n_units : sms;
   const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(k_emit_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const bool f8 = a.map.val_dtype == MR_FP8_E4M3;
+  auto kern = f8 ? k_emit_tc<true> : k_emit_tc<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps(kKEmitTc, a.stream);
-  k_emit_tc<<<grid, kThreads, smem, a.stream>>>(tq, tk, p);
+  kern<<<grid, kThreads, smem, a.stream>>>(tq, tk, p);
   return cudaGetLastError();
 }
 

@@ -18,6 +18,7 @@ struct CompressArgs {
   WsHeader* ws;
   float* lse_ws;    // [H][L] natural-log row normaliser (workspace)
   int* count_ws;    // [H * nqb]
+  int qb0, qb1;     // query blocks processed: qb0 <= I < qb1
   mr_bsr map;
   cudaStream_t stream;
 };
@@ -27,11 +28,14 @@ struct RetrieveArgs {
   const float* W;
   int H_r;
   const void* V;
+  int64_t v_elems;  // elements of the V allocation: every value read stays below it
   void* O;
   mr_dtype dt;
   int d_v, n_req;
   const int64_t* v_req_off;
   int64_t v_req_stride, v_head_stride;
+  int v_group;      // receiver heads per value head
+  int qb0, qb1;     // output query blocks: qb0 <= I < qb1
   WsHeader* ws;
   cudaStream_t stream;
 };
@@ -65,10 +69,15 @@ cudaError_t tc_compress_stats(const CompressArgs& a);  // row normalisers, masse
 cudaError_t tc_emit(const CompressArgs& a);            // kept tiles -> map storage
 bool tc_retrieve_supported(const RetrieveArgs& a);
 cudaError_t tc_retrieve(const RetrieveArgs& a);
+bool tc_dense_supported(const DenseArgs& a);
+cudaError_t tc_dense(const DenseArgs& a);
 
 // Shared by every compress path: exclusive scan of the kept counts into row_ptr, nnz, capacity.
 cudaError_t launch_scan_counts(const int* count, int n, mr_bsr map, WsHeader* ws, cudaStream_t st);
 
 cudaError_t launch_export(const mr_bsr& map, int64_t n_tiles, float* out, cudaStream_t st);
+
+// Measurement: the retrieval's map reads alone (each kept tile moved to shared memory `readers` times).
+cudaError_t launch_gather_probe(const mr_bsr& map, int readers, WsHeader* ws, cudaStream_t st);
 
 }  // namespace mr

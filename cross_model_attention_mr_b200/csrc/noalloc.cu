@@ -56,3 +56,11 @@ extern "C" mr_status mr_compress_noalloc(const void* Q, const void* K, mr_dtype 
   return mr_compress(Q, K, dt, H_s, L, d, scale, p, bias, out, scratch,
                      (size_t)MR_COMPRESS_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+extern "C" mr_status mr_compress_noalloc_status(void* stream) {
+  void* scratch = nullptr;
+  const mr_status s = scratch_address(&scratch);
+  if (s != MR_OK) return s;
+  // the scratch begins with the status header that the last call's kernels wrote
+  return mr_sync_status(scratch, stream);
+}

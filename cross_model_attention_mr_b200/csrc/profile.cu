@@ -13,7 +13,7 @@ namespace {
 
 const char* const kNames[kNumKernelIds] = {
     "mr_compress_stats", "mr_scan_counts", "mr_emit", "mr_retrieve", "mr_dense", "mr_export",
-    "mr_compress_tc", "mr_emit_tc", "mr_retrieve_tc", "mr_dense_tc", "mr_wait_probe", "mr_prep",
+    "mr_compress_tc", "mr_emit_tc", "mr_retrieve_tc", "mr_dense_tc", "mr_wait_probe", "mr_prep", "mr_gather_probe",
 };
 
 struct Record {

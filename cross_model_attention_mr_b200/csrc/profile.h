@@ -17,7 +17,8 @@ enum KernelId {
   kKDenseTc = 9,
   kKWaitProbe = 10,
   kKPrep = 11,
-  kNumKernelIds = 12
+  kKGatherProbe = 12,
+  kNumKernelIds = 13
 };
 
 // Called immediately before and after each kernel launch on `st`.

@@ -22,6 +22,8 @@
 // Every wait is bounded; a wait that runs out records MR_ERR_TIMEOUT and the CTA drains its
 // in-flight copies and MMAs, frees Tensor Memory and returns.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -58,13 +60,19 @@ struct Params {
   const uint32_t* kept_bits;
   const int32_t* row_ptr;
   const __nv_bfloat16* vals;
+  const uint8_t* vals8;      // fp8 (e4m3) maps
+  const float* tile_scale;   // fp8 maps: one scale per 32-row x 64-key piece
   int64_t capacity;
   const float* W;
   __nv_bfloat16* O;
   const int64_t* v_req_off;
   int64_t v_req_stride, v_head_stride;
+  int64_t v_rows;  // rows of 128 values in the V allocation (the tensor map's extent)
+  int v_group;     // receiver heads per value head
   int H_s, H_r, L, B, nqb, nkw, n_req;
   int R, n_hg, n_rg, n_rb, n_units;
+  int rb_hi;       // 128-row blocks rb_hi - n_rb .. rb_hi - 1 hold the output query blocks
+  int qb0, qb1;    // output query blocks qb0 <= I < qb1
   int per;      // units per row block: head groups x request groups
   int groups;   // > 0: grouped schedule with this many groups of `per` CTAs (one wave)
   uint32_t* progress;  // [gridDim.x] pages consumed by each CTA's mixers (workspace, zeroed)
@@ -85,10 +93,18 @@ struct Page {
 };
 constexpr uint32_t kUnitEnd = 1u, kEmptyUnit = 2u, kEnd = 4u;
 
-struct Smem {
+// fp8 maps: one 16-key piece of one row per thread and panel (a 64-key panel row is 64 bytes), and
+// the piece's scale next to it; values are mixed in half precision pre-scaled by 2^14 (so they stay
+// in its normal range; a mixed value is at most 2^14), undone exactly in the epilogue.
+constexpr int kPieces8 = 1;
+constexpr float kF8Pre = 16384.f;
+
+template <bool F8>
+struct SmemT {
   __nv_bfloat16 x[kAcc][128 * 64];
   __nv_bfloat16 v[kAcc][64 * 128];
-  uint4 ring[kQueue][2][kPieces][kMixThreads];  // [pair slot][entry of the pair][piece][mixer thread]
+  uint4 ring[kQueue][2][F8 ? kPieces8 : kPieces][kMixThreads];  // [pair slot][entry][piece][mixer thread]
+  float sring[kQueue][2][F8 ? kMixThreads : 1];                  // fp8: each entry's piece scale
   Page page[kPages];
   uint64_t plan_full[kPages], plan_empty[kPages];
   uint64_t x_full, x_empty, v_full, v_empty, o_full, o_empty, mma_done;
@@ -103,19 +119,19 @@ struct Unit {
 __device__ __forceinline__ Unit decode(const Params& p, int k) {
   const int per = p.n_hg * p.n_rg;
   Unit u;
-  u.rb = p.n_rb - 1 - k / per;
+  u.rb = p.rb_hi - 1 - k / per;
   const int rest = k % per;
   u.hg = rest % p.n_hg;
   u.rg = rest / p.n_hg;
+  // query blocks of the unit outside the output range are -1 (no entries, no rows written)
   if (p.B == 128) {
     u.I0 = u.rb;
     u.I1 = -1;
-    u.Jmax = u.rb;
   } else {
-    u.I0 = 2 * u.rb;
-    u.I1 = (2 * u.rb + 1 < p.nqb) ? 2 * u.rb + 1 : -1;
-    u.Jmax = u.I1 >= 0 ? u.I1 : u.I0;
+    u.I0 = 2 * u.rb >= p.qb0 ? 2 * u.rb : -1;
+    u.I1 = (2 * u.rb + 1 < p.qb1) ? 2 * u.rb + 1 : -1;
   }
+  u.Jmax = u.I1 >= 0 ? u.I1 : u.I0;
   return u;
 }
 
@@ -134,9 +150,9 @@ __device__ __forceinline__ int units_of_cta(const Params& p) {
 __device__ __forceinline__ Unit unit_at(const Params& p, int t) {
   if (p.groups > 0) {
     const int g = blockIdx.x / p.per, m = blockIdx.x % p.per;
-    const int rb = p.n_rb - 1 - (g + p.groups * t);
+    const int rb = p.rb_hi - 1 - (g + p.groups * t);
     // (rb, hg, rg) -> the index decode() maps back to the same unit
-    return decode(p, (p.n_rb - 1 - rb) * p.per + m);
+    return decode(p, (p.rb_hi - 1 - rb) * p.per + m);
   }
   return decode(p, (int)blockIdx.x + t * (int)gridDim.x);
 }
@@ -160,7 +176,8 @@ __device__ __forceinline__ bool acc_valid(const Params& p, const Unit& u, int G,
   return u.hg * G + g < p.H_r && u.rg * p.R + q < p.n_req;
 }
 
-__device__ __forceinline__ void fail(Smem& s, const Params& p, uint32_t detail) {
+template <typename S>
+__device__ __forceinline__ void fail(S& s, const Params& p, uint32_t detail) {
   set_status(p.ws, MR_ERR_TIMEOUT, detail);
   s.abort = 1;
 }
@@ -198,8 +215,8 @@ struct RowCursor {
 // ------------------------------------------------------------------------------------------------
 // Planner warp: pages (one per sub-step, plus a marker after every unit and one at the end).  It
 // waits only for page slots, never for the tensor core.
-template <int G>
-__device__ void planner(Smem& s, const Params& p) {
+template <int G, bool F8>
+__device__ void planner(SmemT<F8>& s, const Params& p) {
   const int lane = threadIdx.x & 31;
   uint32_t np = 0;    // pages written
   const int nparts = p.B / 64;
@@ -306,9 +323,14 @@ __device__ void planner(Smem& s, const Params& p) {
                 const int64_t tt = cur[pt][hs].first + cur[pt][hs].count;
                 if (tt < p.capacity) {
                   t = (uint32_t)tt;
-                  const char* src = reinterpret_cast<const char*>(p.vals + tt * (int64_t)p.B * p.B) +
-                                    (p.B == 128 ? 16384 * h : 0);
-                  bulk_prefetch_l2(src, p.B == 128 ? 16384u : 8192u);
+                  if (F8) {
+                    const char* src = reinterpret_cast<const char*>(p.vals8 + tt * (int64_t)p.B * p.B) + 64 * p.B * h;
+                    bulk_prefetch_l2(src, 64u * (uint32_t)p.B);
+                  } else {
+                    const char* src = reinterpret_cast<const char*>(p.vals + tt * (int64_t)p.B * p.B) +
+                                      (p.B == 128 ? 16384 * h : 0);
+                    bulk_prefetch_l2(src, p.B == 128 ? 16384u : 8192u);
+                  }
                 } else {
                   set_status(p.ws, MR_ERR_CAPACITY, 3u);  // the map overflowed: this tile was never stored
                 }
@@ -382,8 +404,8 @@ struct SubWalker {
   }
 };
 
-template <int G>
-__device__ void issue_v(Smem& s, const Params& p, const CUtensorMap* tmap_v, const Unit& u, int j0) {
+template <int G, typename S>
+__device__ void issue_v(S& s, const Params& p, const CUtensorMap* tmap_v, const Unit& u, int j0) {
   uint32_t bytes = 0;
   for (int a = 0; a < G * p.R; ++a)
     if (acc_valid(p, u, G, a)) bytes += 64 * 128 * 2;
@@ -391,17 +413,24 @@ __device__ void issue_v(Smem& s, const Params& p, const CUtensorMap* tmap_v, con
   for (int a = 0; a < G * p.R; ++a) {
     if (!acc_valid(p, u, G, a)) continue;
     const int r = u.hg * G + a / p.R, q = u.rg * p.R + a % p.R;
-    const int64_t off = (p.v_req_off ? p.v_req_off[q] : (int64_t)q * p.v_req_stride) + (int64_t)r * p.v_head_stride;
-    const int row = (int)(off / 128) + j0;
-    tma_load_2d(&s.v[a][0], tmap_v, &s.v_full, 0, row);
-    tma_load_2d(&s.v[a][64 * 64], tmap_v, &s.v_full, 64, row);
+    const int64_t off = (p.v_req_off ? p.v_req_off[q] : (int64_t)q * p.v_req_stride) +
+                        (int64_t)(r / p.v_group) * p.v_head_stride;
+    // a request's rows must start on a row of the tensor map and end inside the allocation; if
+    // not, load from past the map's extent (TMA fills zeros) and record the bad offset
+    int64_t row = off / 128 + j0;
+    if (off < 0 || (off & 127) != 0 || off / 128 + (int64_t)p.L > p.v_rows) {
+      set_status(p.ws, MR_ERR_DEVICE_CHECK, 5u);
+      row = p.v_rows;
+    }
+    tma_load_2d(&s.v[a][0], tmap_v, &s.v_full, 0, (int)row);
+    tma_load_2d(&s.v[a][64 * 64], tmap_v, &s.v_full, 64, (int)row);
   }
 }
 
 // MMA warp: per sub-step, X (from the mixers) x V (loaded here one sub-step ahead) into the unit's
 // accumulators; the next V load is issued once these MMAs have read the buffer.
-template <int G>
-__device__ void mma_issuer(Smem& s, const Params& p, const CUtensorMap* tmap_v) {
+template <int G, bool F8>
+__device__ void mma_issuer(SmemT<F8>& s, const Params& p, const CUtensorMap* tmap_v) {
   const int lane = threadIdx.x & 31;
   const uint32_t idesc = idesc_bf16_f32(128, 128, false, true);
   const uint32_t tbase = s.tmem_base;
@@ -496,10 +525,23 @@ __device__ void mma_issuer(Smem& s, const Params& p, const CUtensorMap* tmap_v) 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ float lds32f(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+// two e4m3 values (low byte = lower column) -> half2
+__device__ __forceinline__ __half2 e4m3x2_to_half2(uint32_t two) {
+  const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
+  return *reinterpret_cast<const __half2*>(&r);
 }
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
@@ -512,14 +554,22 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 // l % 8 of the 128-byte-swizzled
 // panel row: eight consecutive keys 8 * ((l % 8) ^ (a_k % 8)).  X is written with the same
 // swizzle, so the thread writes its chunks back to the positions it read them from.
-template <int G>
-__device__ void mixers(Smem& s, const Params& p) {
+template <int G, bool F8>
+__device__ void mixers(SmemT<F8>& s, const Params& p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int half = p.B == 64 ? (warp / (kMixWarps / 2)) : 0;  // 64-key blocks: which of the unit's two query blocks
   const uint32_t rowb = (uint32_t)(kRowsW * warp + (lane >> 3));
   const uint32_t my_off = (p.B == 64 ? (rowb & 63u) : rowb) * 128u + (uint32_t)(lane & 7) * 16u;  // bytes
   const uint32_t tile_bytes = (uint32_t)(p.B * p.B * 2);
   const char* vals = reinterpret_cast<const char*>(p.vals);
+  // fp8 maps: thread (w, l) owns row rowb8 = 8 w + l / 4 of the unit and the 16-key piece l % 4 of
+  // each 64-byte panel row, and fetches the scale of the 32-row x 64-key piece it falls in
+  const uint32_t rowb8 = (uint32_t)(kRowsW * warp + (lane >> 2));
+  const uint32_t trow8 = p.B == 64 ? (rowb8 & 63u) : rowb8;
+  const uint32_t my_off8 = trow8 * 64u + (uint32_t)(lane & 3) * 16u;
+  const uint32_t sc_row8 = (trow8 >> 5) * (uint32_t)(p.B / 64);
+  const uint32_t nsc = (uint32_t)fp8_scales_per_tile(p.B);
+  const char* vals8 = reinterpret_cast<const char*>(p.vals8);
   const uint32_t tbase = s.tmem_base;
   const int tw = warp & 3;  // Tensor Memory lane quadrant of this warp
 
@@ -567,11 +617,25 @@ __device__ void mixers(Smem& s, const Params& p) {
   // there is nothing to copy, so group counts stay aligned with pairs); the move to the
   // following page is taken lazily, at the next call
   const uint32_t ring0 = smem_u32(&s.ring[0][0][0][threadIdx.x]);
-  constexpr uint32_t kPiece = kMixThreads * 16u, kEntry = kPieces * kPiece, kSlot = 2u * kEntry;
+  constexpr int kPc = F8 ? kPieces8 : kPieces;
+  constexpr uint32_t kPiece = kMixThreads * 16u, kEntry = kPc * kPiece, kSlot = 2u * kEntry;
+  const uint32_t sring0 = smem_u32(&s.sring[0][0][F8 ? threadIdx.x : 0]);
+  constexpr uint32_t kSEntry = kMixThreads * 4u, kSSlot = 2u * kSEntry;
   auto fetch = [&](uint32_t slot) -> bool {
     bool good = true;
     if (!f_done && ef == nf) good = fetch_seek(pf + 1);
-    if (good && !f_done) {
+    if (good && !f_done && F8) {
+      const uint32_t tt[2] = {fpg->e[2 * ef].t[half], fpg->e[2 * ef + 1].t[half]};
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        if (tt[j] == kNone) continue;
+        const uint64_t t = tt[j];
+        cp_async16(ring0 + slot * kSlot + j * kEntry,
+                   vals8 + (t * (uint64_t)(p.B * p.B) + hf * 64u * (uint32_t)p.B + my_off8));
+        cp_async4(sring0 + slot * kSSlot + j * kSEntry, p.tile_scale + (t * nsc + sc_row8 + hf));
+      }
+      ++ef;
+    } else if (good && !f_done) {
       const uint32_t t0 = fpg->e[2 * ef].t[half], t1 = fpg->e[2 * ef + 1].t[half];
       const uint32_t dst = ring0 + slot * kSlot;
       const uint32_t panel = hf * 16384u + my_off;
@@ -593,10 +657,33 @@ __device__ void mixers(Smem& s, const Params& p) {
 
   constexpr int kW = 4 * kPieces;  // packed bf16 pairs per thread per panel
   float2 acc[G][kW];               // fp32 accumulators for columns (2e, 2e + 1) of the thread's chunks
+  __half2 acch[G][8];              // fp8 maps: half accumulators of the thread's 16 keys (x 2^14)
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
-    for (int e = 0; e < kW; ++e) acc[g][e] = make_float2(0.f, 0.f);
+    for (int e = 0; e < kW; ++e) {
+      acc[g][e] = make_float2(0.f, 0.f);
+      acch[g][e] = __float2half2_rn(0.f);
+    }
+
+  // fp8 entry: acch[g] += (W[r_g, s] * scale * 2^14) * (the thread's 16 e4m3 values)
+  auto mix_entry8 = [&](const Entry& E, uint32_t data, uint32_t sdata) {
+    const float sc = lds32f(sdata) * kF8Pre;
+    __half2 w2[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) w2[g] = __float2half2_rn(E.w[g] * sc);
+    const uint4 d = lds128(data);
+    const uint32_t wd[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __half2 lo = e4m3x2_to_half2(wd[e]), hi = e4m3x2_to_half2(wd[e] >> 16);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        acch[g][2 * e] = __hfma2(w2[g], lo, acch[g][2 * e]);
+        acch[g][2 * e + 1] = __hfma2(w2[g], hi, acch[g][2 * e + 1]);
+      }
+    }
+  };
 
   // one entry: acc[g] += W[r_g, s] * (this thread's 16 values of the sender head's panel)
   auto mix_entry = [&](const Entry& E, uint32_t data) {
@@ -625,7 +712,24 @@ __device__ void mixers(Smem& s, const Params& p) {
   auto hand_x = [&]() -> bool {
     if (nsub > 0 && !mbar_wait(&s.x_empty, (nsub - 1) & 1, &s.abort, kTimeoutNs)) return false;
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
+    for (int g = 0; g < (F8 ? G : 0); ++g) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {  // the thread's two 8-key chunks of X row rowb8
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 a = __half22float2(acch[g][4 * c + e]);
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(a.x, a.y);
+          pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
+          acch[g][4 * c + e] = __float2half2_rn(0.f);
+        }
+        const uint32_t lc = 2u * (uint32_t)(lane & 3) + (uint32_t)c;
+        char* xb = reinterpret_cast<char*>(&s.x[g][0]) + rowb8 * 128 + ((lc ^ (rowb8 & 7u)) << 4);
+        *reinterpret_cast<uint4*>(xb) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < (F8 ? 0 : G); ++g) {
 #pragma unroll
       for (int k = 0; k < kPieces; ++k) {
         uint32_t pk[4];
@@ -653,6 +757,9 @@ __device__ void mixers(Smem& s, const Params& p) {
     const Unit u = unit_at(p, nunit);
     const int row = 32 * tw + lane;
     const int i = u.rb * 128 + row;
+    const int qblk = p.B == 128 ? u.rb : 2 * u.rb + (row >> 6);
+    const bool row_out = i < p.L && qblk >= p.qb0 && qblk < p.qb1;  // rows outside the range stay as they are
+    const float osc = F8 ? 1.f / kF8Pre : 1.f;                       // fp8 maps were mixed x 2^14
 #pragma unroll 1
     for (int a = warp >> 2; a < G * p.R; a += kMixWarps / 4) {
       const bool valid = acc_valid(p, u, G, a);
@@ -663,14 +770,14 @@ __device__ void mixers(Smem& s, const Params& p) {
         uint32_t v[16];
         tmem_ld16(tbase + ((uint32_t)(32 * tw) << 16) + 128 * a + 16 * cc, v);
         tmem_wait_ld();
-        if (valid && i < p.L) {
+        if (valid && row_out) {
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             uint32_t pk[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float x0 = any ? __uint_as_float(v[8 * c + 2 * e]) : 0.f;
-              const float x1 = any ? __uint_as_float(v[8 * c + 2 * e + 1]) : 0.f;
+              const float x0 = any ? __uint_as_float(v[8 * c + 2 * e]) * osc : 0.f;
+              const float x1 = any ? __uint_as_float(v[8 * c + 2 * e + 1]) * osc : 0.f;
               const __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
               pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
             }
@@ -720,7 +827,12 @@ __device__ void mixers(Smem& s, const Params& p) {
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       const Entry& E = cpg->e[2 * ec + j];
-      if (E.t[half] != kNone) mix_entry(E, data + j * kEntry);
+      if (E.t[half] != kNone) {
+        if (F8)
+          mix_entry8(E, data + j * kEntry, sring0 + slot * kSSlot + j * kSEntry);
+        else
+          mix_entry(E, data + j * kEntry);
+      }
     }
     if (++ec == nc) {
       // end of the sub-step: hand X to the tensor core, release the page, run any markers
@@ -743,10 +855,10 @@ __device__ void mixers(Smem& s, const Params& p) {
   if (!good) fail(s, p, 0x301);
 }
 
-template <int G>
+template <int G, bool F8>
 __global__ void __launch_bounds__(kThreads, 1) k_retrieve_tc(const __grid_constant__ CUtensorMap tmap_v, Params p) {
   extern __shared__ unsigned char smem_raw[];
-  Smem& s = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+  SmemT<F8>& s = *reinterpret_cast<SmemT<F8>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kPages; ++i) {
@@ -771,33 +883,40 @@ __global__ void __launch_bounds__(kThreads, 1) k_retrieve_tc(const __grid_consta
   __syncthreads();
   tc_fence_after();
   if (warp < kMixWarps)
-    mixers<G>(s, p);
+    mixers<G, F8>(s, p);
   else if (warp == kPlanWarp)
-    planner<G>(s, p);
+    planner<G, F8>(s, p);
   else
-    mma_issuer<G>(s, p, &tmap_v);
+    mma_issuer<G, F8>(s, p, &tmap_v);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == kMmaWarp) tmem_dealloc(s.tmem_base, 512);
 }
 
-template <int G>
+template <int G, bool F8>
 cudaError_t launch_g(const RetrieveArgs& a, const Params& p, const CUtensorMap& tm, int grid, cudaStream_t st) {
-  const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(k_retrieve_tc<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = sizeof(SmemT<F8>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(k_retrieve_tc<G, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps(kKRetrieveTc, st);
-  k_retrieve_tc<G><<<grid, kThreads, smem, st>>>(tm, p);
+  k_retrieve_tc<G, F8><<<grid, kThreads, smem, st>>>(tm, p);
   return cudaGetLastError();
+}
+
+template <bool F8>
+cudaError_t launch_any(const RetrieveArgs& a, const Params& p, const CUtensorMap& tm, int grid, int G) {
+  if (G == 4) return launch_g<4, F8>(a, p, tm, grid, a.stream);
+  if (G == 2) return launch_g<2, F8>(a, p, tm, grid, a.stream);
+  return launch_g<1, F8>(a, p, tm, grid, a.stream);
 }
 
 }  // namespace
 
 bool tc_retrieve_supported(const RetrieveArgs& a) {
-  return a.dt == MR_BF16 && a.d_v == 128 && (a.map.block == 64 || a.map.block == 128) && a.map.H_s <= 64 &&
+  return a.dt == MR_BF16 && (a.map.val_dtype == MR_BF16 || a.map.val_dtype == MR_FP8_E4M3) && a.d_v == 128 && (a.map.block == 64 || a.map.block == 128) && a.map.H_s <= 64 &&
          a.map.capacity_tiles < (int64_t)kNone && a.v_head_stride % 128 == 0 &&
-         (a.v_req_off != nullptr || a.v_req_stride % 128 == 0);
+         (a.v_req_off != nullptr || a.v_req_stride % 128 == 0) && a.v_elems / 128 < ((int64_t)1 << 31) - 1;
 }
 
 cudaError_t tc_retrieve(const RetrieveArgs& a) {
@@ -805,12 +924,16 @@ cudaError_t tc_retrieve(const RetrieveArgs& a) {
   p.kept_bits = a.map.kept_bits;
   p.row_ptr = a.map.row_ptr;
   p.vals = (const __nv_bfloat16*)a.map.vals;
+  p.vals8 = (const uint8_t*)a.map.vals;
+  p.tile_scale = a.map.tile_scale;
   p.capacity = a.map.capacity_tiles;
   p.W = a.W;
   p.O = (__nv_bfloat16*)a.O;
   p.v_req_off = a.v_req_off;
   p.v_req_stride = a.v_req_stride;
   p.v_head_stride = a.v_head_stride;
+  p.v_rows = a.v_elems / 128;
+  p.v_group = a.v_group;
   p.H_s = a.map.H_s;
   p.H_r = a.H_r;
   p.L = a.map.L;
@@ -818,6 +941,8 @@ cudaError_t tc_retrieve(const RetrieveArgs& a) {
   p.nqb = a.map.L / a.map.block;
   p.nkw = (p.nqb + 31) / 32;
   p.n_req = a.n_req;
+  p.qb0 = a.qb0;
+  p.qb1 = a.qb1;
   int G = 4;
   if (a.n_req >= 4)
     G = 1;
@@ -826,20 +951,18 @@ cudaError_t tc_retrieve(const RetrieveArgs& a) {
   p.R = kAcc / G;
   p.n_hg = (a.H_r + G - 1) / G;
   p.n_rg = (a.n_req + p.R - 1) / p.R;
-  p.n_rb = (a.map.L + 127) / 128;
+  // 128-row blocks holding the output query blocks
+  const int rb_lo = p.B == 128 ? a.qb0 : a.qb0 / 2;
+  p.rb_hi = p.B == 128 ? a.qb1 : (a.qb1 + 1) / 2;
+  p.n_rb = p.rb_hi - rb_lo;
   p.n_units = p.n_rb * p.n_hg * p.n_rg;
   p.per = p.n_hg * p.n_rg;
   p.ws = a.ws;
   p.progress = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(a.ws) + kWsHeaderBytes);
-  // V viewed as rows of 128 bf16; rows are addressed from the request offset and head stride.
-  // With strided requests the exact extent is known (rows past it read as zeros); with a device
-  // offset table it is not, and the view spans the 32-bit row range.
+  // V viewed as rows of 128 bf16 spanning exactly the caller's allocation: rows past it read as
+  // zeros, and offsets are checked against it on the device
   CUtensorMap tm;
-  uint64_t rows = ((uint64_t)1 << 31) - 1;
-  if (a.v_req_off == nullptr)
-    rows = (uint64_t)(((int64_t)(a.n_req - 1) * a.v_req_stride + (int64_t)(a.H_r - 1) * a.v_head_stride) / 128) +
-           (uint64_t)a.map.L;
-  if (!make_tmap_bf16_2d(&tm, a.V, 128, rows, 256, 64, 64)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tm, a.V, 128, (uint64_t)p.v_rows, 256, 64, 64)) return cudaErrorInvalidValue;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -852,9 +975,8 @@ cudaError_t tc_retrieve(const RetrieveArgs& a) {
     grid = p.n_units < sms ? p.n_units : sms;
     if (grid > kMaxProgressCtas) grid = kMaxProgressCtas;  // one progress counter per CTA
   }
-  if (G == 4) return launch_g<4>(a, p, tm, grid, a.stream);
-  if (G == 2) return launch_g<2>(a, p, tm, grid, a.stream);
-  return launch_g<1>(a, p, tm, grid, a.stream);
+  if (a.map.val_dtype == MR_FP8_E4M3) return launch_any<true>(a, p, tm, grid, G);
+  return launch_any<false>(a, p, tm, grid, G);
 }
 
 }  // namespace mr

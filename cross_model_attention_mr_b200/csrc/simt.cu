@@ -6,6 +6,7 @@
 // block, receiver head, request) output tile for retrieval, and a (sequence tile, head) for dense
 // attention.  Work units with more causal tiles are scheduled first (larger query blocks first).
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -73,7 +74,7 @@ template <typename T, int BLK, int D>
 __global__ void __launch_bounds__(kThreads) k_compress_stats(
     const T* __restrict__ Q, const T* __restrict__ K, int H, int L, float scale, float p, Bias bias,
     float* __restrict__ lse_ws, int* __restrict__ count_ws, uint32_t* __restrict__ kept_bits,
-    float* __restrict__ kept_mass, float* __restrict__ mass_out, float* __restrict__ lse_out) {
+    float* __restrict__ kept_mass, float* __restrict__ mass_out, float* __restrict__ lse_out, int qb_hi) {
   extern __shared__ float smem[];
   float* Qs = smem;
   float* Ks = Qs + BLK * (D + 1);
@@ -86,7 +87,7 @@ __global__ void __launch_bounds__(kThreads) k_compress_stats(
   __shared__ int kstar_s;
 
   const int nqb = L / BLK, nkb = nqb, nkw = (nkb + 31) / 32;
-  const int I = nqb - 1 - (int)(blockIdx.x / H);
+  const int I = qb_hi - 1 - (int)(blockIdx.x / H);  // query blocks qb_hi - 1, qb_hi - 2, ...
   const int h = (int)(blockIdx.x % H);
   const int u = h * nqb + I;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
@@ -205,13 +206,13 @@ __global__ void __launch_bounds__(kThreads) k_emit(
     const T* __restrict__ Q, const T* __restrict__ K, int H, int L, float scale, Bias bias,
     const float* __restrict__ lse_ws, const int32_t* __restrict__ row_ptr,
     const uint32_t* __restrict__ kept_bits, int64_t capacity, int32_t* __restrict__ col_idx,
-    TV* __restrict__ vals) {
+    TV* __restrict__ vals, int qb_hi) {
   extern __shared__ float smem[];
   float* Qs = smem;
   float* Ks = Qs + BLK * (D + 1);
   __shared__ float lse_s[BLK];
   const int nqb = L / BLK, nkw = (nqb + 31) / 32;
-  const int I = nqb - 1 - (int)(blockIdx.x / H);
+  const int I = qb_hi - 1 - (int)(blockIdx.x / H);  // query blocks qb_hi - 1, qb_hi - 2, ...
   const int h = (int)(blockIdx.x % H);
   const int u = h * nqb + I;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
@@ -247,35 +248,66 @@ __global__ void __launch_bounds__(kThreads) k_emit(
   }
 }
 
+// Stored map values: element at storage offset `off` of tile t, as fp32, with its tile coordinates.
+template <typename TM>
+struct MapVals {
+  const TM* vals;
+  const float* scale;  // fp8 only
+  __device__ __forceinline__ float at(int64_t t, int off, int B) const { return to_f32(vals[t * B * B + off]); }
+  __device__ __forceinline__ void coords(int off, int B, int& a, int& b) const { tile_coords<TM>(off, B, a, b); }
+};
+template <>
+struct MapVals<uint8_t> {
+  const uint8_t* vals;
+  const float* scale;
+  __device__ __forceinline__ void coords(int off, int B, int& a, int& b) const {
+    const int panel = off / (B * 64), rem = off - panel * B * 64;
+    a = rem >> 6;
+    b = panel * 64 + (rem & 63);
+  }
+  __device__ __forceinline__ float at(int64_t t, int off, int B) const {
+    int a, b;
+    coords(off, B, a, b);
+    const __half_raw h = __nv_cvt_fp8_to_halfraw(vals[t * B * B + off], __NV_E4M3);
+    return __half2float(*reinterpret_cast<const __half*>(&h)) * scale[t * fp8_scales_per_tile(B) + fp8_scale_index(a, b, B)];
+  }
+};
+
 // ---------------------------------------------------------------------------------------------
 // Retrieval: O_r[I] = sum_{J <= I} X[I,J] V_r[J],  X = sum_s W[r,s] A_s[I,J] over kept tiles.
 // One CTA per (query block, receiver head, request).  X is built in shared memory only.
 // ---------------------------------------------------------------------------------------------
-template <typename T, int BLK, int DV>
+template <typename T, typename TM, int BLK, int DV>
 __global__ void __launch_bounds__(kThreads) k_retrieve(
     const int32_t* __restrict__ row_ptr, const uint32_t* __restrict__ kept_bits,
-    const T* __restrict__ vals, int64_t capacity, int H_s, int L, const float* __restrict__ W,
-    int H_r, const T* __restrict__ V, T* __restrict__ O, const int64_t* __restrict__ v_req_off,
-    int64_t v_req_stride, int64_t v_head_stride, WsHeader* ws) {
+    MapVals<TM> mv, int64_t capacity, int H_s, int L, const float* __restrict__ W,
+    int H_r, const T* __restrict__ V, int64_t v_elems, T* __restrict__ O,
+    const int64_t* __restrict__ v_req_off, int64_t v_req_stride, int64_t v_head_stride, int v_group,
+    int qb_hi, WsHeader* ws) {
   extern __shared__ float smem[];
   float* Xs = smem;                   // [BLK][BLK + 1]
   float* Vs = Xs + BLK * (BLK + 1);   // [BLK][DV + 1]
   __shared__ float Ws[64];
   const int nqb = L / BLK, nkw = (nqb + 31) / 32;
-  const int I = nqb - 1 - (int)(blockIdx.x / H_r);
+  const int I = qb_hi - 1 - (int)(blockIdx.x / H_r);
   const int r = (int)(blockIdx.x % H_r);
   const int q = blockIdx.y;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   constexpr int R = BLK / 16, C = DV / 16, E = BLK * BLK / kThreads;
   for (int s = tid; s < H_s; s += kThreads) Ws[s] = W[(size_t)r * H_s + s];
-  const T* Vr = V + (v_req_off ? v_req_off[q] : (int64_t)q * v_req_stride) + (int64_t)r * v_head_stride;
+  // value head r / v_group of request q; rows 0 .. (I + 1) * BLK - 1 must lie inside the allocation,
+  // else the request reads zeros and the status word records the bad offset
+  const int64_t voff = (v_req_off ? v_req_off[q] : (int64_t)q * v_req_stride) + (int64_t)(r / v_group) * v_head_stride;
+  const bool v_ok = voff >= 0 && voff + (int64_t)(I + 1) * BLK * DV <= v_elems;
+  if (!v_ok && tid == 0) set_status(ws, MR_ERR_DEVICE_CHECK, 4u);
+  const T* Vr = V + (v_ok ? voff : 0);
   float acc[R][C];
 #pragma unroll
   for (int a = 0; a < R; ++a)
 #pragma unroll
     for (int c = 0; c < C; ++c) acc[a][c] = 0.f;
   __syncthreads();
-  for (int J = 0; J <= I; ++J) {
+  for (int J = 0; J <= (v_ok ? I : -1); ++J) {
     float x[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) x[e] = 0.f;
@@ -290,17 +322,16 @@ __global__ void __launch_bounds__(kThreads) k_retrieve(
         continue;
       }
       any = true;
-      const T* tile = vals + (size_t)t * BLK * BLK;
       const float w = Ws[s];
 #pragma unroll
-      for (int e = 0; e < E; ++e) x[e] = fmaf(w, to_f32(tile[tid + e * kThreads]), x[e]);
+      for (int e = 0; e < E; ++e) x[e] = fmaf(w, mv.at(t, tid + e * kThreads, BLK), x[e]);
     }
     if (!any) continue;
     __syncthreads();
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       int ra, cb;
-      tile_coords<T>(tid + e * kThreads, BLK, ra, cb);
+      mv.coords(tid + e * kThreads, BLK, ra, cb);
       Xs[ra * (BLK + 1) + cb] = x[e];
     }
     load_rows<T, BLK, DV>(Vs, Vr + (size_t)J * BLK * DV, BLK);
@@ -486,6 +517,18 @@ __global__ void k_export(const TV* __restrict__ vals, int64_t n_elems, int B, fl
   }
 }
 
+// fp8 tiles: e4m3 value times the scale of its 32-row x 64-key piece
+__global__ void k_export_fp8(const uint8_t* __restrict__ vals, const float* __restrict__ scale, int64_t n_elems,
+                             int B, float* __restrict__ out) {
+  const int64_t tsz = (int64_t)B * B;
+  const MapVals<uint8_t> mv{vals, scale};
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n_elems; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = e / tsz;
+    const int w = (int)(e - t * tsz);
+    out[e] = mv.at(t, tile_offset_fp8(w / B, w % B, B), B);
+  }
+}
+
 template <typename KernelT>
 cudaError_t set_smem(KernelT k, size_t bytes) {
   return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
@@ -500,9 +543,9 @@ cudaError_t compress_impl(const CompressArgs& a) {
   if (e != cudaSuccess) return e;
   {
     ProfScope ps(kKCompressStats, a.stream);
-    k1<<<a.H * nqb, kThreads, smem, a.stream>>>(
+    k1<<<a.H * (a.qb1 - a.qb0), kThreads, smem, a.stream>>>(
         (const T*)a.Q, (const T*)a.K, a.H, a.L, a.scale, a.p, a.bias, a.lse_ws, a.count_ws,
-        a.map.kept_bits, a.map.kept_mass, a.map.mass, a.map.lse);
+        a.map.kept_bits, a.map.kept_mass, a.map.mass, a.map.lse, a.qb1);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = launch_scan_counts(a.count_ws, a.H * nqb, a.map, a.ws, a.stream)) != cudaSuccess) return e;
@@ -510,40 +553,38 @@ cudaError_t compress_impl(const CompressArgs& a) {
   if ((e = set_smem(k3, smem)) != cudaSuccess) return e;
   {
     ProfScope ps(kKEmit, a.stream);
-    k3<<<a.H * nqb, kThreads, smem, a.stream>>>(
+    k3<<<a.H * (a.qb1 - a.qb0), kThreads, smem, a.stream>>>(
         (const T*)a.Q, (const T*)a.K, a.H, a.L, a.scale, a.bias, a.lse_ws, a.map.row_ptr,
-        a.map.kept_bits, a.map.capacity_tiles, a.map.col_idx, (TV*)a.map.vals);
+        a.map.kept_bits, a.map.capacity_tiles, a.map.col_idx, (TV*)a.map.vals, a.qb1);
   }
   return cudaGetLastError();
 }
 
 template <typename T, typename TV, int BLK, int D>
 cudaError_t emit_impl(const CompressArgs& a) {
-  const int nqb = a.L / BLK;
   const size_t smem = (size_t)2 * BLK * (D + 1) * sizeof(float);
   auto k3 = k_emit<T, TV, BLK, D>;
   cudaError_t e = set_smem(k3, smem);
   if (e != cudaSuccess) return e;
   ProfScope ps(kKEmit, a.stream);
-  k3<<<a.H * nqb, kThreads, smem, a.stream>>>(
+  k3<<<a.H * (a.qb1 - a.qb0), kThreads, smem, a.stream>>>(
       (const T*)a.Q, (const T*)a.K, a.H, a.L, a.scale, a.bias, a.lse_ws, a.map.row_ptr,
-      a.map.kept_bits, a.map.capacity_tiles, a.map.col_idx, (TV*)a.map.vals);
+      a.map.kept_bits, a.map.capacity_tiles, a.map.col_idx, (TV*)a.map.vals, a.qb1);
   return cudaGetLastError();
 }
 
-template <typename T, int BLK, int DV>
+template <typename T, typename TM, int BLK, int DV>
 cudaError_t retrieve_impl(const RetrieveArgs& a) {
-  const int nqb = a.map.L / BLK;
   const size_t smem = (size_t)(BLK * (BLK + 1) + BLK * (DV + 1)) * sizeof(float);
-  auto k = k_retrieve<T, BLK, DV>;
+  auto k = k_retrieve<T, TM, BLK, DV>;
+  const MapVals<TM> mv{(const TM*)a.map.vals, a.map.tile_scale};
   cudaError_t e = set_smem(k, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(nqb * a.H_r, a.n_req);
+  dim3 grid((a.qb1 - a.qb0) * a.H_r, a.n_req);
   ProfScope ps(kKRetrieve, a.stream);
-  k<<<grid, kThreads, smem, a.stream>>>(a.map.row_ptr, a.map.kept_bits, (const T*)a.map.vals,
-                                         a.map.capacity_tiles, a.map.H_s, a.map.L, a.W, a.H_r,
-                                         (const T*)a.V, (T*)a.O, a.v_req_off, a.v_req_stride,
-                                         a.v_head_stride, a.ws);
+  k<<<grid, kThreads, smem, a.stream>>>(a.map.row_ptr, a.map.kept_bits, mv, a.map.capacity_tiles, a.map.H_s, a.map.L, a.W, a.H_r,
+                                         (const T*)a.V, a.v_elems, (T*)a.O, a.v_req_off, a.v_req_stride,
+                                         a.v_head_stride, a.v_group, a.qb1, a.ws);
   return cudaGetLastError();
 }
 
@@ -590,10 +631,17 @@ cudaError_t simt_emit(const CompressArgs& a) {
 cudaError_t simt_retrieve(const RetrieveArgs& a) {
   const bool bf = a.dt == MR_BF16;
   const int B = a.map.block;
-  if (B == 64 && a.d_v == 64) return bf ? retrieve_impl<__nv_bfloat16, 64, 64>(a) : retrieve_impl<float, 64, 64>(a);
-  if (B == 64 && a.d_v == 128) return bf ? retrieve_impl<__nv_bfloat16, 64, 128>(a) : retrieve_impl<float, 64, 128>(a);
-  if (B == 128 && a.d_v == 64) return bf ? retrieve_impl<__nv_bfloat16, 128, 64>(a) : retrieve_impl<float, 128, 64>(a);
-  if (B == 128 && a.d_v == 128) return bf ? retrieve_impl<__nv_bfloat16, 128, 128>(a) : retrieve_impl<float, 128, 128>(a);
+  if (a.map.val_dtype == MR_FP8_E4M3) {  // bf16 values, fp8 map
+    if (B == 64 && a.d_v == 64) return retrieve_impl<__nv_bfloat16, uint8_t, 64, 64>(a);
+    if (B == 64 && a.d_v == 128) return retrieve_impl<__nv_bfloat16, uint8_t, 64, 128>(a);
+    if (B == 128 && a.d_v == 64) return retrieve_impl<__nv_bfloat16, uint8_t, 128, 64>(a);
+    if (B == 128 && a.d_v == 128) return retrieve_impl<__nv_bfloat16, uint8_t, 128, 128>(a);
+    return cudaErrorInvalidValue;
+  }
+  if (B == 64 && a.d_v == 64) return bf ? retrieve_impl<__nv_bfloat16, __nv_bfloat16, 64, 64>(a) : retrieve_impl<float, float, 64, 64>(a);
+  if (B == 64 && a.d_v == 128) return bf ? retrieve_impl<__nv_bfloat16, __nv_bfloat16, 64, 128>(a) : retrieve_impl<float, float, 64, 128>(a);
+  if (B == 128 && a.d_v == 64) return bf ? retrieve_impl<__nv_bfloat16, __nv_bfloat16, 128, 64>(a) : retrieve_impl<float, float, 128, 64>(a);
+  if (B == 128 && a.d_v == 128) return bf ? retrieve_impl<__nv_bfloat16, __nv_bfloat16, 128, 128>(a) : retrieve_impl<float, float, 128, 128>(a);
   return cudaErrorInvalidValue;
 }
 
@@ -612,7 +660,9 @@ cudaError_t launch_export(const mr_bsr& map, int64_t n_tiles, float* out, cudaSt
   if (n == 0) return cudaSuccess;
   const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
   ProfScope ps(kKExport, st);
-  if (map.val_dtype == MR_BF16)
+  if (map.val_dtype == MR_FP8_E4M3)
+    k_export_fp8<<<blocks, 256, 0, st>>>((const uint8_t*)map.vals, map.tile_scale, n, map.block, out);
+  else if (map.val_dtype == MR_BF16)
     k_export<__nv_bfloat16><<<blocks, 256, 0, st>>>((const __nv_bfloat16*)map.vals, n, map.block, out);
   else
     k_export<float><<<blocks, 256, 0, st>>>((const float*)map.vals, n, map.block, out);

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmr.so")
 
 MR_OK, MR_ERR_INVALID_ARG, MR_ERR_UNSUPPORTED, MR_ERR_CAPACITY = 0, 1, 2, 3
 MR_ERR_CUDA, MR_ERR_TIMEOUT, MR_ERR_DEVICE_CHECK, MR_ERR_RANGE = 4, 5, 6, 7
-MR_BF16, MR_F32 = 0, 1
+MR_BF16, MR_F32, MR_FP8_E4M3 = 0, 1, 2
 
 _c_i32, _c_i64, _c_f32, _c_p, _c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 
@@ -30,10 +30,15 @@ class LogitBias(ctypes.Structure):
                 ("kb_bias", _c_p), ("kb_block", _c_i32), ("n_kb", _c_i32)]
 
 
+class RetrieveOpts(ctypes.Structure):
+    _fields_ = [("qb_begin", _c_i32), ("qb_end", _c_i32), ("v_group", _c_i32)]
+
+
 class BSR(ctypes.Structure):
     _fields_ = [("H_s", _c_i32), ("L", _c_i32), ("block", _c_i32), ("val_dtype", ctypes.c_int),
                 ("capacity_tiles", _c_i64), ("row_ptr", _c_p), ("col_idx", _c_p), ("vals", _c_p),
-                ("kept_mass", _c_p), ("kept_bits", _c_p), ("mass", _c_p), ("lse", _c_p), ("nnz", _c_p)]
+                ("kept_mass", _c_p), ("kept_bits", _c_p), ("mass", _c_p), ("lse", _c_p), ("nnz", _c_p),
+                ("tile_scale", _c_p)]
 
 
 EXPORTS = {
@@ -44,11 +49,16 @@ EXPORTS = {
     "mr_bsr_max_tiles": ([ctypes.c_int] * 3, _c_i64),
     "mr_compress": ([_c_p, _c_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _c_f32, _c_f32,
                      ctypes.POINTER(LogitBias), ctypes.POINTER(BSR), _c_p, _c_sz, _c_p], ctypes.c_int),
+    "mr_compress_blocks": ([_c_p, _c_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _c_f32, _c_f32,
+                            ctypes.POINTER(LogitBias), ctypes.c_int, ctypes.c_int, ctypes.POINTER(BSR), _c_p, _c_sz,
+                            _c_p], ctypes.c_int),
     "mr_compress_noalloc": ([_c_p, _c_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _c_f32, _c_f32,
                              ctypes.POINTER(LogitBias), ctypes.POINTER(BSR), _c_p], ctypes.c_int),
+    "mr_compress_noalloc_status": ([_c_p], ctypes.c_int),
     "mr_retrieve_workspace_bytes": ([ctypes.POINTER(BSR), ctypes.c_int, ctypes.c_int, ctypes.c_int], _c_sz),
-    "mr_retrieve": ([ctypes.POINTER(BSR), _c_p, ctypes.c_int, _c_p, _c_p, ctypes.c_int, ctypes.c_int,
-                     ctypes.c_int, _c_p, _c_i64, _c_i64, _c_p, _c_sz, _c_p], ctypes.c_int),
+    "mr_retrieve": ([ctypes.POINTER(BSR), _c_p, ctypes.c_int, _c_p, _c_i64, _c_p, ctypes.c_int, ctypes.c_int,
+                     ctypes.c_int, _c_p, _c_i64, _c_i64, ctypes.POINTER(RetrieveOpts), _c_p, _c_sz, _c_p],
+                    ctypes.c_int),
     "mr_dense_ref_workspace_bytes": ([ctypes.c_int], _c_sz),
     "mr_dense_ref": ([_c_p, _c_p, _c_p, _c_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                       _c_p, _c_p, _c_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _c_f32,
@@ -56,6 +66,15 @@ EXPORTS = {
     "mr_sync_status": ([_c_p, _c_p], ctypes.c_int),
     "mr_bsr_nnz": ([ctypes.POINTER(BSR), ctypes.POINTER(_c_i64), _c_p], ctypes.c_int),
     "mr_bsr_export": ([ctypes.POINTER(BSR), _c_i64, _c_p, _c_p], ctypes.c_int),
+    "mr_bm_create": ([ctypes.c_int, _c_i64], _c_p),
+    "mr_bm_destroy": ([_c_p], None),
+    "mr_bm_insert": ([_c_p, _c_p, ctypes.c_int, ctypes.POINTER(BSR), ctypes.c_int, _c_i64], _c_i64),
+    "mr_bm_lookup": ([_c_p, _c_p, ctypes.c_int, ctypes.POINTER(_c_i64)], ctypes.c_int),
+    "mr_bm_map": ([_c_p, _c_i64, ctypes.c_int, ctypes.POINTER(BSR)], ctypes.c_int),
+    "mr_bm_release": ([_c_p, _c_i64], ctypes.c_int),
+    "mr_bm_evicted": ([_c_p, ctypes.POINTER(_c_i64), ctypes.c_int], ctypes.c_int),
+    "mr_bm_stats": ([_c_p, ctypes.POINTER(_c_i64)], ctypes.c_int),
+    "mr_gather_probe": ([ctypes.POINTER(BSR), ctypes.c_int, _c_p, _c_sz, _c_p], ctypes.c_int),
     "mr_profile_enable": ([ctypes.c_int], ctypes.c_int),
     "mr_profile_read": ([_c_p, _c_p, ctypes.c_int], ctypes.c_int),
     "mr_kernel_name": ([ctypes.c_int], ctypes.c_char_p),
@@ -97,7 +116,12 @@ def _dt(t: torch.Tensor) -> int:
 
 
 def _torch_dtype(dt: int):
-    return torch.bfloat16 if dt == MR_BF16 else torch.float32
+    return {MR_BF16: torch.bfloat16, MR_F32: torch.float32, MR_FP8_E4M3: torch.uint8}[dt]
+
+
+def fp8_scales_per_tile(block: int) -> int:
+    """Scales of an fp8 tile: one per 32-row x 64-key piece."""
+    return (block // 32) * (block // 64)
 
 
 def _stream(stream) -> Optional[int]:
@@ -168,10 +192,13 @@ class Map:
         self.mass = torch.zeros((n, self.nqb), dtype=torch.float32, device=dev) if store_mass else None
         self.lse = torch.zeros((H_s, L), dtype=torch.float32, device=dev) if store_lse else None
         self.nnz = torch.zeros(1, dtype=torch.int64, device=dev)
+        self.tile_scale = (torch.zeros((max(1, self.capacity), fp8_scales_per_tile(block)), dtype=torch.float32,
+                                       device=dev) if dtype == MR_FP8_E4M3 else None)
         self.c = BSR(H_s, L, block, dtype, self.capacity, self.row_ptr.data_ptr(), self.col_idx.data_ptr(),
                      self.vals.data_ptr(), self.kept_mass.data_ptr(), self.kept_bits.data_ptr(),
                      self.mass.data_ptr() if self.mass is not None else None,
-                     self.lse.data_ptr() if self.lse is not None else None, self.nnz.data_ptr())
+                     self.lse.data_ptr() if self.lse is not None else None, self.nnz.data_ptr(),
+                     self.tile_scale.data_ptr() if self.tile_scale is not None else None)
 
     def nnz_host(self, stream=None) -> int:
         v = _c_i64(0)
@@ -203,6 +230,8 @@ def _map_arrays(m: "Map", n_stored: int):
         # bf16 travels as its bit pattern, so every backend moves it unchanged
         vals = m.vals[:n_stored]
         arrays += [m.col_idx[:n_stored], vals.view(torch.int16) if vals.dtype == torch.bfloat16 else vals]
+        if m.tile_scale is not None:
+            arrays.append(m.tile_scale[:n_stored])
     return arrays
 
 
@@ -235,6 +264,55 @@ def recv_map(src: int, device="cuda", group=None) -> "Map":
     return m
 
 
+# ------------------------------------------------------------------------------------------------
+# One sequence split across ranks by query-block range (MapFlow section 6: distributed settings).
+# Compression units (head, query block) and retrieval rows are independent once every key and
+# value row up to the range's end is present, so the only exchange is an all-gather of the
+# ranks' K and V row shards; maps and outputs stay on their rank.
+# ------------------------------------------------------------------------------------------------
+def split_query_blocks(nqb: int, world: int, align: int = 1):
+    """Contiguous ranges [(qb_begin, qb_end)] of the nqb query blocks, one per rank, balanced by
+    causal work (query block I costs I + 1 key blocks).  Cuts fall on multiples of ``align``
+    (2 for block 64, whose kernels work on pairs of query blocks); a rank may get an empty range
+    when there are fewer aligned pieces than ranks."""
+    if nqb < 1 or world < 1 or align < 1:
+        raise ValueError("need nqb, world, align >= 1")
+    cum = np.concatenate([[0.0], np.cumsum(np.arange(1, nqb + 1, dtype=np.float64))])  # work before cut c
+    total = cum[-1]
+    cands = sorted(set(list(range(0, nqb + 1, align)) + [nqb]))
+    cuts = [0]
+    for r in range(1, world):
+        target = total * r / world
+        # the aligned cut whose prefix work is closest to the target, never before the previous cut
+        best = min((c for c in cands if c >= cuts[-1]), key=lambda c: abs(cum[c] - target))
+        cuts.append(best)
+    cuts.append(nqb)
+    return [(cuts[r], cuts[r + 1]) for r in range(world)]
+
+
+def row_shards(L: int, ranges, block: int):
+    """Token rows [(row_begin, row_end)] of each rank's query-block range."""
+    return [(q0 * block, q1 * block) for q0, q1 in ranges]
+
+
+def gather_row_shards(local: torch.Tensor, shards, group=None) -> torch.Tensor:
+    """All-gather of per-rank row shards [H][rows_r][d] into the full [H][L][d] on every rank
+    (torch.distributed: NCCL between GPUs, gloo between CPU ranks).  Shards are padded to the
+    longest one so every rank sends the same number of bytes."""
+    import torch.distributed as dist
+    H, _, d = local.shape
+    longest = max(e - b for b, e in shards)
+    L = shards[-1][1]
+    pad = torch.zeros((H, longest, d), dtype=local.dtype, device=local.device)
+    pad[:, : local.shape[1]] = local
+    parts = [torch.empty_like(pad) for _ in shards]
+    dist.all_gather(parts, pad.contiguous(), group=group)
+    full = torch.empty((H, L, d), dtype=local.dtype, device=local.device)
+    for (b, e), part in zip(shards, parts):
+        full[:, b:e] = part[:, : e - b]
+    return full
+
+
 def max_tiles(H_s: int, L: int, block: int) -> int:
     return int(LIB.mr_bsr_max_tiles(H_s, L, block))
 
@@ -245,8 +323,11 @@ def compress_workspace_bytes(H_s, L, d, block) -> int:
 
 def compress(Q: torch.Tensor, K: torch.Tensor, p: float, block: int, bias: Optional[Bias] = None,
              scale: Optional[float] = None, capacity: Optional[int] = None, out: Optional[Map] = None,
-             ws: Optional[Workspace] = None, store_mass=False, store_lse=False, stream=None) -> Map:
-    """mr_compress: Q, K [H_s][L][d] (bf16 or fp32, CUDA) -> Map."""
+             ws: Optional[Workspace] = None, store_mass=False, store_lse=False, stream=None,
+             blocks: Optional[tuple] = None, map_dtype: Optional[int] = None) -> Map:
+    """mr_compress: Q, K [H_s][L][d] (bf16 or fp32, CUDA) -> Map.  ``blocks=(qb_begin, qb_end)``
+    calls mr_compress_blocks: only those query blocks, the other rows of the map left empty.
+    ``map_dtype=MR_FP8_E4M3`` stores e4m3 values with per-piece scales (bf16 inputs)."""
     _need_cuda(Q, K)
     H, L, d = Q.shape
     dt = _dt(Q)
@@ -254,12 +335,17 @@ def compress(Q: torch.Tensor, K: torch.Tensor, p: float, block: int, bias: Optio
         scale = 1.0 / math.sqrt(d)
     if out is None:
         cap = max_tiles(H, L, block) if capacity is None else capacity
-        out = Map(H, L, block, dt, cap, Q.device, store_mass, store_lse)
+        out = Map(H, L, block, dt if map_dtype is None else map_dtype, cap, Q.device, store_mass, store_lse)
     if ws is None:
         ws = Workspace(compress_workspace_bytes(H, L, d, block), Q.device)
     out.ws = ws
-    check(LIB.mr_compress(Q.data_ptr(), K.data_ptr(), dt, H, L, d, float(scale), float(p), _bias_ptr(bias),
-                          ctypes.byref(out.c), ws.ptr, ws.nbytes, _stream(stream)), "mr_compress")
+    if blocks is None:
+        check(LIB.mr_compress(Q.data_ptr(), K.data_ptr(), dt, H, L, d, float(scale), float(p), _bias_ptr(bias),
+                              ctypes.byref(out.c), ws.ptr, ws.nbytes, _stream(stream)), "mr_compress")
+    else:
+        check(LIB.mr_compress_blocks(Q.data_ptr(), K.data_ptr(), dt, H, L, d, float(scale), float(p),
+                                     _bias_ptr(bias), int(blocks[0]), int(blocks[1]), ctypes.byref(out.c), ws.ptr,
+                                     ws.nbytes, _stream(stream)), "mr_compress_blocks")
     return out
 
 
@@ -270,9 +356,12 @@ def retrieve_workspace_bytes(m: Map, H_r: int, d_v: int, n_req: int) -> int:
 def retrieve(m: Map, W: torch.Tensor, V: torch.Tensor, out: Optional[torch.Tensor] = None,
              v_req_off: Optional[torch.Tensor] = None, v_req_stride: Optional[int] = None,
              v_head_stride: Optional[int] = None, n_req: Optional[int] = None,
-             ws: Optional[Workspace] = None, stream=None) -> torch.Tensor:
-    """mr_retrieve: W [H_r][H_s] fp32; V [H_r][L][d_v] or [n_req][H_r][L][d_v] (or a packed buffer
-    with explicit strides/offsets) -> O [n_req][H_r][L][d_v]."""
+             ws: Optional[Workspace] = None, stream=None, blocks: Optional[tuple] = None,
+             v_group: int = 1, v_elems: Optional[int] = None) -> torch.Tensor:
+    """mr_retrieve: W [H_r][H_s] fp32; V [H_v][L][d_v] or [n_req][H_v][L][d_v] (or a packed buffer
+    with explicit strides/offsets), H_v = H_r / v_group -> O [n_req][H_r][L][d_v].
+    ``blocks=(qb_begin, qb_end)`` writes only those query blocks' rows of O; ``v_elems`` defaults to
+    the number of elements of V."""
     _need_cuda(W, V, v_req_off)
     H_r = W.shape[0]
     dt = _dt(V)
@@ -282,15 +371,21 @@ def retrieve(m: Map, W: torch.Tensor, V: torch.Tensor, out: Optional[torch.Tenso
     if n_req is None:
         n_req = V.shape[0] if V.dim() == 4 else 1
     if v_req_stride is None:
-        v_req_stride = H_r * v_head_stride
+        v_req_stride = (H_r // max(1, v_group)) * v_head_stride
+    if v_elems is None:
+        v_elems = V.numel()
     if out is None:
         out = torch.empty((n_req, H_r, m.L, d_v), dtype=V.dtype, device=V.device)
     _need_cuda(out)
     if ws is None:
         ws = Workspace(retrieve_workspace_bytes(m, H_r, d_v, n_req), V.device)
-    check(LIB.mr_retrieve(ctypes.byref(m.c), W.data_ptr(), H_r, V.data_ptr(), out.data_ptr(), dt, d_v, n_req,
-                          v_req_off.data_ptr() if v_req_off is not None else None, int(v_req_stride),
-                          int(v_head_stride), ws.ptr, ws.nbytes, _stream(stream)), "mr_retrieve")
+    opts = None
+    if blocks is not None or v_group != 1:
+        b = blocks if blocks is not None else (0, 0)
+        opts = ctypes.byref(RetrieveOpts(int(b[0]), int(b[1]), int(v_group)))
+    check(LIB.mr_retrieve(ctypes.byref(m.c), W.data_ptr(), H_r, V.data_ptr(), int(v_elems), out.data_ptr(), dt,
+                          d_v, n_req, v_req_off.data_ptr() if v_req_off is not None else None, int(v_req_stride),
+                          int(v_head_stride), opts, ws.ptr, ws.nbytes, _stream(stream)), "mr_retrieve")
     return out
 
 
@@ -317,6 +412,13 @@ def dense_ref(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, cu_q: torch.Ten
     return out
 
 
+def gather_probe(m: "Map", readers: int, ws: Optional[Workspace] = None, stream=None) -> None:
+    """mr_gather_probe: the retrieval's map reads alone (measurement)."""
+    if ws is None:
+        ws = Workspace(256, m.vals.device)
+    check(LIB.mr_gather_probe(ctypes.byref(m.c), int(readers), ws.ptr, ws.nbytes, _stream(stream)), "mr_gather_probe")
+
+
 def profile_enable(on: bool = True) -> bool:
     return bool(LIB.mr_profile_enable(1 if on else 0))
 
@@ -336,3 +438,90 @@ def profile_read() -> dict:
 
 def kernel_launches() -> int:
     return int(LIB.mr_kernel_launches())
+
+
+def compress_noalloc(Q: torch.Tensor, K: torch.Tensor, p: float, out: Map, bias: Optional[Bias] = None,
+                     scale: Optional[float] = None, stream=None) -> Map:
+    """mr_compress_noalloc: as compress, with the library's fixed scratch instead of a workspace."""
+    _need_cuda(Q, K)
+    H, L, d = Q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    check(LIB.mr_compress_noalloc(Q.data_ptr(), K.data_ptr(), _dt(Q), H, L, d, float(scale), float(p),
+                                  _bias_ptr(bias), ctypes.byref(out.c), _stream(stream)), "mr_compress_noalloc")
+    return out
+
+
+def compress_noalloc_status(stream=None) -> int:
+    """mr_compress_noalloc_status: device status of the last allocation-free compression."""
+    return int(LIB.mr_compress_noalloc_status(_stream(stream)))
+
+
+
+class BlockManager:
+    """mr_bm_*: prefix-hash index from token prefixes to stored maps (MapFlow section 5.3).
+
+    ``insert(tokens, maps)`` registers the per-layer maps of one sequence (the Map objects are kept
+    alive here until their entry is evicted and collected by ``collect_evicted``);
+    ``lookup(tokens)`` returns (reusable query blocks, entry id); ``map(entry, layer)`` gives a Map
+    view to pass to ``retrieve(..., blocks=(0, k))``."""
+
+    def __init__(self, block: int, budget_bytes: int = 0):
+        self.h = LIB.mr_bm_create(int(block), int(budget_bytes))
+        if not self.h:
+            raise MRError(MR_ERR_INVALID_ARG, "mr_bm_create")
+        self.block = block
+        self._maps = {}
+
+    def __del__(self):
+        if getattr(self, "h", None):
+            LIB.mr_bm_destroy(self.h)
+            self.h = None
+
+    def insert(self, tokens, maps, map_bytes: Optional[int] = None) -> int:
+        tok = np.ascontiguousarray(tokens, dtype=np.int32)
+        arr = (BSR * len(maps))(*[m.c for m in maps])
+        if map_bytes is None:
+            map_bytes = sum(m.vals.numel() * m.vals.element_size() for m in maps)
+        eid = int(LIB.mr_bm_insert(self.h, tok.ctypes.data_as(_c_p), int(tok.shape[0]), arr, len(maps),
+                                   int(map_bytes)))
+        if eid < 0:
+            raise MRError(-eid, "mr_bm_insert")
+        self._maps[eid] = list(maps)
+        return eid
+
+    def lookup(self, tokens):
+        tok = np.ascontiguousarray(tokens, dtype=np.int32)
+        e = _c_i64(-1)
+        k = int(LIB.mr_bm_lookup(self.h, tok.ctypes.data_as(_c_p), int(tok.shape[0]), ctypes.byref(e)))
+        if k < 0:
+            raise MRError(-k, "mr_bm_lookup")
+        return k, int(e.value)
+
+    def map(self, entry: int, layer: int) -> "Map":
+        d = BSR()
+        check(LIB.mr_bm_map(self.h, int(entry), int(layer), ctypes.byref(d)), "mr_bm_map")
+        m = self._maps[entry][layer]
+        assert m.c.vals == d.vals  # the descriptor is the registered map's
+        return m
+
+    def release(self, entry: int) -> None:
+        check(LIB.mr_bm_release(self.h, int(entry)), "mr_bm_release")
+
+    def collect_evicted(self):
+        """Ids evicted since the last call; their Map objects (device arrays) are dropped here."""
+        ids = (_c_i64 * 64)()
+        out = []
+        while True:
+            n = int(LIB.mr_bm_evicted(self.h, ids, 64))
+            out += [int(ids[i]) for i in range(n)]
+            if n < 64:
+                break
+        for i in out:
+            self._maps.pop(i, None)
+        return out
+
+    def stats(self) -> dict:
+        v = (_c_i64 * 5)()
+        check(LIB.mr_bm_stats(self.h, v), "mr_bm_stats")
+        return dict(zip(("entries", "bytes", "lookups", "hits", "hit_blocks"), [int(x) for x in v]))

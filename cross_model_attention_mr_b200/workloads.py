@@ -187,13 +187,12 @@ class Layer:
     bias: Bias
 
 
-def draw_layers(spec: Spec, layers: Optional[List[int]] = None) -> List[Layer]:
-    """Draw the requested layers (all by default), consuming the stream in layer order."""
-    want = set(range(spec.n_layers) if layers is None else layers)
+def iter_layers(spec: Spec):
+    """Yield every layer of the workload in order, drawn from one stream (the same values as
+    draw_layers), so a caller can move each layer to the device before the next is drawn."""
     rng = np.random.default_rng(spec.seed)
     n_kb = spec.L // spec.block
-    out: List[Layer] = []
-    for layer in range(max(want) + 1):
+    for _ in range(spec.n_layers):
         Q = np.empty((spec.H_s, spec.L, spec.d), np.float32)
         K = np.empty_like(Q)
         for h in range(spec.H_s):
@@ -204,8 +203,18 @@ def draw_layers(spec: Spec, layers: Optional[List[int]] = None) -> List[Layer]:
         for r in range(spec.H_r):
             V[r] = _normal(rng, (spec.L, spec.d_v), 1.0, spec.dtype)
         W = _W(spec, rng)
+        yield Layer(Q=Q, K=K, V=V, W=W, bias=bias)
+
+
+def draw_layers(spec: Spec, layers: Optional[List[int]] = None) -> List[Layer]:
+    """Draw the requested layers (all by default), consuming the stream in layer order."""
+    want = set(range(spec.n_layers) if layers is None else layers)
+    out: List[Layer] = []
+    for layer, lay in enumerate(iter_layers(spec)):
         if layer in want:
-            out.append(Layer(Q=Q, K=K, V=V, W=W, bias=bias))
+            out.append(lay)
+        if layer >= max(want):
+            break
     return out
 
 

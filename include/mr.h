@@ -46,7 +46,13 @@ typedef enum {
   MR_ERR_RANGE = 7         /* a row's logits span too wide a range for the fp32 exponent path */
 } mr_status;
 
-typedef enum { MR_BF16 = 0, MR_F32 = 1 } mr_dtype;
+/*
+ * Element types.  MR_FP8_E4M3 is a map value type only (inputs stay MR_BF16): MapFlow section 9,
+ * "Compact representations for reusable attention state".  An fp8 map stores each value as e4m3
+ * (IEEE-style, 4 exponent bits with bias 7, 3 mantissa bits) times a float scale per 32-row x 64-key
+ * piece of a tile (mr_bsr.tile_scale).
+ */
+typedef enum { MR_BF16 = 0, MR_F32 = 1, MR_FP8_E4M3 = 2 } mr_dtype;
 
 /*
  * Synthetic causal logit bias b(h, i, j), added to sigma * q_i.k_j for j <= i.  It stands in for
@@ -85,12 +91,19 @@ typedef struct {
  *             chunk position c ^ (a % 8).  So element (a, b) sits at
  *               (b / P) * block * P + a * P + E * (((b % P) / E) ^ (a % 8)) + b % E,
  *             E = 16 / sizeof(element).  (Each panel is a 128-byte-swizzled MMA operand.)
+ *             MR_FP8_E4M3 tiles are stored in panels of 64 columns, each panel holding its `block`
+ *             rows of 64 bytes in turn with no swizzle: element (a, b) at
+ *               (b / 64) * block * 64 + a * 64 + b % 64,
+ *             and the value is e4m3(a, b) * tile_scale[t * S + (a / 32) * (block / 64) + b / 64],
+ *             S = (block / 32) * (block / 64) scales per tile.
  *             mr_bsr_export converts tiles to plain row-major fp32.
  *   kept_mass float  [H_s * nqb]      mass of the kept blocks (fp64 sum, rounded to fp32)
  *   kept_bits uint32 [H_s * nqb][nkb_words]  bit (J % 32) of word J / 32 set iff block J kept
  *   mass      float  [H_s * nqb][nkb] optional block masses (NULL = not written); J > I is 0
  *   lse       float  [H_s][L]         optional natural-log row normaliser log(sum_j exp(s_ij))
  *   nnz       int64  [1]              number of kept tiles (may exceed capacity_tiles)
+ *   tile_scale float [capacity_tiles][S]  MR_FP8_E4M3 maps only (else unused, may be NULL): the
+ *             scale of each 32-row x 64-key piece, max(piece) / 448 (448 = largest e4m3 value)
  */
 typedef struct {
   int32_t H_s;
@@ -106,6 +119,7 @@ typedef struct {
   float* mass;
   float* lse;
   int64_t* nnz;
+  float* tile_scale;
 } mr_bsr;
 
 /* Library version (major * 100 + minor). */
@@ -141,7 +155,10 @@ int64_t mr_bsr_max_tiles(int H_s, int L, int block);
  *   out    map descriptor (see mr_bsr); out->H_s, L, block must equal the arguments.
  *   ws     workspace of at least mr_compress_workspace_bytes(H_s, L, d, block) bytes.
  * Supported: d in {64, 128}; block in {64, 128}; L a positive multiple of block with
- * L / block <= 256; H_s <= 64.  MR_BF16 maps use bf16 vals; MR_F32 maps use fp32 vals.
+ * L / block <= 256; H_s <= 64.  MR_BF16 maps use bf16 vals; MR_F32 maps use fp32 vals; bf16 inputs
+ * with d = 128 may also write an MR_FP8_E4M3 map (out->val_dtype = MR_FP8_E4M3, out->tile_scale
+ * set), whose values carry the e4m3 rounding error (at most 2^-4 relative, plus 2^-10 of their
+ * piece's scale below the normal range).
  * bf16 with d = 128 (and per-key-block biases, if any, on multiples of 32 keys) runs on the
  * tensor-core kernels; other shapes on the CUDA-core kernels.  Either way vals hold the tiles in
  * the 128-byte-panel layout described at mr_bsr.
@@ -151,6 +168,20 @@ int64_t mr_bsr_max_tiles(int H_s, int L, int block);
 mr_status mr_compress(const void* Q, const void* K, mr_dtype dt, int H_s, int L, int d,
                       float scale, float p, const mr_logit_bias* bias, mr_bsr* out, void* ws,
                       size_t ws_bytes, void* stream);
+
+/*
+ * mr_compress restricted to the query blocks qb_begin <= I < qb_end of every head (all heads, all
+ * key blocks J <= I): MapFlow section 6 ("Chunked Prefill"), and the per-rank share of one sequence
+ * split across GPUs by query-block range.  Rows of *out outside the range are written as empty
+ * (count 0, no kept bits, kept mass 0); their row_ptr entries repeat the running total, so the
+ * map is a valid BSR map of the whole layer whose only non-empty rows are the range's.  Row
+ * normalisers in out->lse are written for the range's rows (and, for block 64, possibly for the
+ * other block of a 128-row pair).  Needs the same workspace as mr_compress.  Requires
+ * 0 <= qb_begin < qb_end <= L / block; mr_compress is this call with the full range.
+ */
+mr_status mr_compress_blocks(const void* Q, const void* K, mr_dtype dt, int H_s, int L, int d,
+                             float scale, float p, const mr_logit_bias* bias, int qb_begin,
+                             int qb_end, mr_bsr* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Allocation-free variant of mr_compress.  The paper has no counterpart: this is a deployment
@@ -176,13 +207,23 @@ mr_status mr_compress(const void* Q, const void* K, mr_dtype dt, int H_s, int L,
  *     parts that must start at zero, in stream order.  Calls whose work can overlap on the GPU
  *     (other streams or other host threads without ordering between them) race on the array and
  *     corrupt each other's maps: order them.
- *   - There is no caller-visible workspace, so mr_sync_status cannot read this call's status
- *     word.  A map that outgrew its capacity shows as *out->nnz > out->capacity_tiles.
+ *   - There is no caller-visible workspace: read the status word of the most recent call with
+ *     mr_compress_noalloc_status (capacity overflow, a bounded wait that ran out).
+ *   - The array's device address is cached per device for the life of its CUDA context; after
+ *     cudaDeviceReset the cached address is stale, so do not call this entry point again in a
+ *     process that reset a device it used.
  */
 #define MR_COMPRESS_NOALLOC_SCRATCH_BYTES (256 + 4194304 + 65536)
 mr_status mr_compress_noalloc(const void* Q, const void* K, mr_dtype dt, int H_s, int L, int d,
                               float scale, float p, const mr_logit_bias* bias, mr_bsr* out,
                               void* stream);
+
+/*
+ * Synchronise `stream` and return the device-side status that the most recent
+ * mr_compress_noalloc call on the current device recorded in the fixed scratch array (MR_OK if
+ * nothing failed).  Calls on other streams without ordering to `stream` may overwrite it.
+ */
+mr_status mr_compress_noalloc_status(void* stream);
 
 /*
  * Workspace bytes mr_retrieve needs (device memory, 256-byte aligned): the status header and one
@@ -193,27 +234,52 @@ mr_status mr_compress_noalloc(const void* Q, const void* K, mr_dtype dt, int H_s
 size_t mr_retrieve_workspace_bytes(const mr_bsr* map, int H_r, int d_v, int n_req);
 
 /*
+ * Options of mr_retrieve (pass NULL for the defaults: every query block, one V head per receiver
+ * head).
+ *   qb_begin, qb_end  compute only the output rows of query blocks qb_begin <= I < qb_end
+ *                     (MapFlow section 6, "Chunked Prefill"; also one rank's share of a sequence
+ *                     split across GPUs).  Output rows outside the range are not written.  Both 0:
+ *                     every query block.  Otherwise 0 <= qb_begin < qb_end <= L / block.
+ *   v_group           receiver heads that share one value head (grouped-query attention): receiver
+ *                     head r reads value head r / v_group.  0 or 1: one value head per receiver
+ *                     head.  H_r must be a multiple of v_group.
+ */
+typedef struct {
+  int32_t qb_begin;
+  int32_t qb_end;
+  int32_t v_group;
+} mr_retrieve_opts;
+
+/*
  * Fused translated retrieval: MapFlow sections 3.3 and 5.4.
  *   O_r[i] = sum_{j <= i} ( sum_s W[r][s] * A_s[i][j] * [key block of j kept for (s, block of i)] )
- *            * V_r[j]
- * for every receiver head r < H_r, query row i < map->L and request q < n_req.  The translated
- * map is formed tile by tile on chip and never written to global memory.
- *   map    a map filled by mr_compress (its vals dtype must equal dt)
- *   W      device fp32 [H_r][H_s], row r = receiver head r's weights over sender heads
- *   V      values in dtype dt: element (q, r, j, c) at
- *          V + v_off(q) + r * v_head_stride + j * d_v + c,
- *          v_off(q) = v_req_off[q] (device int64 array) or q * v_req_stride when v_req_off is NULL
- *   O      output in dtype dt: element (q, r, i, c) at O + q * H_r * L * d_v + (r * L + i) * d_v + c
- *   ws     workspace of at least mr_retrieve_workspace_bytes(map, H_r, d_v, n_req) bytes
+ *            * V_g(r)[j],   g(r) = r / v_group
+ * for every receiver head r < H_r, query row i < map->L (or of the options' query-block range) and
+ * request q < n_req.  The translated map is formed tile by tile on chip and never written to
+ * global memory.
+ *   map     a map filled by mr_compress (its vals dtype equals dt, or is MR_FP8_E4M3 with dt = MR_BF16;
+ *           fp8 maps are mixed in half precision from their e4m3 values)
+ *   W       device fp32 [H_r][H_s], row r = receiver head r's weights over sender heads
+ *   V       values in dtype dt: element (q, g, j, c) of value head g at
+ *           V + v_off(q) + g * v_head_stride + j * d_v + c,
+ *           v_off(q) = v_req_off[q] (device int64 array) or q * v_req_stride when v_req_off is NULL
+ *   v_elems number of elements of the V allocation.  Every value read stays below it: the host
+ *           checks strided layouts before launch (MR_ERR_INVALID_ARG); with a device offset table,
+ *           a request whose rows do not fit inside [0, v_elems) (or, on the tensor-core kernel,
+ *           whose offset is not a multiple of d_v) reads zeros instead and records
+ *           MR_ERR_DEVICE_CHECK in the status word.
+ *   O       output in dtype dt: element (q, r, i, c) at O + q * H_r * L * d_v + (r * L + i) * d_v + c
+ *   opts    NULL or mr_retrieve_opts
+ *   ws      workspace of at least mr_retrieve_workspace_bytes(map, H_r, d_v, n_req) bytes
  * Supported: d_v in {64, 128}; H_r <= 256.  bf16 maps with d_v = 128, block 64 or 128 and
  * H_s <= 64 run on the tensor-core kernel; other shapes on the CUDA-core kernel.
  * Tiles a map could not store (capacity overflow at compression) contribute nothing and set
  * MR_ERR_CAPACITY in the status word.
  */
-mr_status mr_retrieve(const mr_bsr* map, const float* W, int H_r, const void* V, void* O,
-                      mr_dtype dt, int d_v, int n_req, const int64_t* v_req_off,
-                      int64_t v_req_stride, int64_t v_head_stride, void* ws, size_t ws_bytes,
-                      void* stream);
+mr_status mr_retrieve(const mr_bsr* map, const float* W, int H_r, const void* V, int64_t v_elems,
+                      void* O, mr_dtype dt, int d_v, int n_req, const int64_t* v_req_off,
+                      int64_t v_req_stride, int64_t v_head_stride, const mr_retrieve_opts* opts,
+                      void* ws, size_t ws_bytes, void* stream);
 
 /* Workspace bytes mr_dense_ref needs (device memory). */
 size_t mr_dense_ref_workspace_bytes(int n_seq);
@@ -228,7 +294,9 @@ size_t mr_dense_ref_workspace_bytes(int n_seq);
  *               0 .. q_offset[s] + i, and requires q_offset[s] + len_q(s) <= len_k(s)
  *   total_q, total_k  host ints equal to cu_q[n_seq] and cu_k[n_seq] (the per-head row
  *               counts of the packed tensors; total_q also sizes the launch)
- * Supported: d, d_v in {64, 128}.
+ * Supported: d, d_v in {64, 128}.  bf16 with d = d_v = 128 (and per-key-block biases, if any, on
+ * multiples of 32 keys) runs on the tensor-core kernel; other shapes on the CUDA-core kernel.
+ * Requires q_offset[s] + len_q(s) <= len_k(s) (not checked: device arrays).
  */
 mr_status mr_dense_ref(const void* Q, const void* K, const void* V, void* O, mr_dtype dt, int H,
                        int d, int d_v, const int32_t* cu_q, const int32_t* cu_k,
@@ -253,6 +321,59 @@ mr_status mr_bsr_nnz(const mr_bsr* map, int64_t* nnz_host, void* stream);
 mr_status mr_bsr_export(const mr_bsr* map, int64_t n_tiles, float* out, void* stream);
 
 /*
+ * Prefix-hash block manager: MapFlow section 5.3 ("Block Manager") and section 1 (prefix-hash
+ * indexing).  Host-side index from token prefixes to stored compressed maps.
+ *
+ * Row (h, I) of a layer's map depends only on the first (I + 1) * block tokens (the map is
+ * causal), so the maps stored for one sequence serve the first k query blocks of every request
+ * whose first k * block tokens are the same: retrieve those rows with mr_retrieve's query-block
+ * range and compute the rest.  Prefixes are keyed by a chained 64-bit hash per block of tokens
+ * and checked token by token, so a hash collision is never reported as a hit.
+ *
+ * The manager keeps copies of the mr_bsr descriptors, never the device arrays: the caller keeps
+ * an entry's arrays alive until the manager reports the entry evicted (mr_bm_evicted), and frees
+ * them then.  Entries carry reference counts (the insert and each successful lookup take one;
+ * mr_bm_release drops one).  When the bytes of the held entries exceed the budget, the least
+ * recently used entries without references are evicted.  All calls are thread-safe, host-only,
+ * and touch no device memory.
+ */
+typedef struct mr_block_manager mr_block_manager;
+
+/* New manager for maps of `block`-token blocks; budget_bytes 0 = no limit.  NULL on bad
+ * arguments or when host memory runs out. */
+mr_block_manager* mr_bm_create(int block, int64_t budget_bytes);
+void mr_bm_destroy(mr_block_manager* bm);
+
+/*
+ * Register the maps of one sequence: tokens (host int32 [n_tokens]; whole blocks are indexed, a
+ * partial last block is ignored) and one descriptor per layer (host array of n_layers, each with
+ * this block size and L >= the indexed tokens).  map_bytes is what the entry counts against the
+ * budget.  Returns the entry id (>= 0, holding one reference) or -mr_status.
+ */
+int64_t mr_bm_insert(mr_block_manager* bm, const int32_t* tokens, int n_tokens, const mr_bsr* maps,
+                     int n_layers, int64_t map_bytes);
+
+/*
+ * Longest stored prefix of `tokens` in whole blocks: returns k, the number of leading query blocks
+ * whose map rows can be reused (0 = none), and writes the entry that holds them to *entry (-1 when
+ * k = 0), taking a reference on it.  Negative -mr_status on bad arguments.
+ */
+int mr_bm_lookup(mr_block_manager* bm, const int32_t* tokens, int n_tokens, int64_t* entry);
+
+/* Copy of the descriptor of `layer` of an entry. */
+mr_status mr_bm_map(mr_block_manager* bm, int64_t entry, int layer, mr_bsr* out);
+
+/* Drop one reference of an entry (then evict to the budget if needed). */
+mr_status mr_bm_release(mr_block_manager* bm, int64_t entry);
+
+/* Ids of evicted entries not reported yet (oldest first, at most max_ids): their device arrays are
+ * no longer referenced by the manager.  Returns how many were written. */
+int mr_bm_evicted(mr_block_manager* bm, int64_t* ids, int max_ids);
+
+/* out[5] = {entries, bytes held, lookups, lookups that hit, query blocks served by hits}. */
+mr_status mr_bm_stats(mr_block_manager* bm, int64_t* out);
+
+/*
  * Measurement hooks (not part of the method).  When profiling is enabled, every entry point
  * records a CUDA event on its stream before and after each kernel it launches; mr_profile_read
  * waits for the recorded events and reports, per kernel id, the summed elapsed milliseconds and
@@ -263,6 +384,16 @@ int mr_profile_enable(int on);      /* returns the previous state; enabling clea
 int mr_profile_read(double* total_ms, int64_t* launches, int max_ids); /* host arrays; returns ids */
 const char* mr_kernel_name(int id);
 int64_t mr_kernel_launches(void);   /* kernels launched by this library in this process */
+
+/*
+ * Measurement kernel (not part of the method): the retrieval's map reads alone.  Walks `map` in
+ * the retrieval's order (128-row blocks longest first; key blocks J <= I; the kept tile of every
+ * sender head) and moves each stored tile into shared memory `readers` times (by `readers` CTAs
+ * working on the same row block side by side, as the retrieval's receiver-head groups do) with
+ * 16-byte asynchronous copies, doing no arithmetic.  Time it on `stream`; bytes moved =
+ * readers * stored tiles * tile bytes.  ws: at least 256 bytes (status header).
+ */
+mr_status mr_gather_probe(const mr_bsr* map, int readers, void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

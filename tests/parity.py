@@ -7,6 +7,10 @@ Tolerances (stated once, used by every test):
   * block masses: |M_gpu - M_oracle| <= MASS_ATOL (fp32 accumulation of fp32 probabilities);
   * stored probabilities: bf16 |P - A| <= 2^-8 |A| + 1e-6; fp32 |P - A| <= 3e-5 |A| + 1e-9;
   * outputs: max |O_gpu - O_oracle(GPU kept sets)| <= OUT_TOL[dtype] * max |V| (2e-2 bf16, 1e-4 fp32).
+  * fp8 (e4m3) maps: stored values |P - A| <= 2^-4 |A| + 3e-6 (half an e4m3 step relative, plus the
+    subnormal step of a piece whose scale is at most 1/448); outputs within 7e-2 max |V|: each
+    translated value is off by at most 2^-4 of itself (plus bf16 and half-precision rounding, < 2^-8),
+    and a row's translated values sum to at most 1, so |dO| <= (2^-4 + 2^-8) max |V|.
 """
 from __future__ import annotations
 
@@ -18,8 +22,8 @@ from cross_model_attention_mr_b200 import mr
 
 BOUNDARY = 1e-5
 MASS_ATOL = 2e-6
-OUT_TOL = {"bf16": 2e-2, "f32": 1e-4}
-VAL_TOL = {"bf16": (2.0 ** -8, 1e-6), "f32": (3e-5, 1e-9)}
+OUT_TOL = {"bf16": 2e-2, "f32": 1e-4, "fp8": 7e-2}
+VAL_TOL = {"bf16": (2.0 ** -8, 1e-6), "f32": (3e-5, 1e-9), "fp8": (2.0 ** -4, 3e-6)}
 
 
 def dev(x: np.ndarray, dtype: str) -> torch.Tensor:
@@ -70,9 +74,11 @@ def check_selection(M: np.ndarray, kept_o: np.ndarray, kept_g: np.ndarray, p: fl
     return True, len(diff), ""
 
 
-def compare_compress(spec, lay, m: mr.Map, units, n_tiles: int = 12, rng_seed: int = 0):
+def compare_compress(spec, lay, m: mr.Map, units, n_tiles: int = 12, rng_seed: int = 0,
+                     all_tiles: bool = False, val_kind: str = None):
     """Check masses, selection, row normalisers and stored values of the given units (h*nqb + I)
-    against the oracle.  Returns a dict of statistics."""
+    against the oracle: every tile both sides kept when ``all_tiles``, else ``n_tiles`` sampled ones
+    (plus a diagonal tile and a J = 0 tile).  Returns a dict of statistics."""
     B = spec.block
     nqb = spec.L // B
     p = p32(spec.p)
@@ -102,39 +108,54 @@ def compare_compress(spec, lay, m: mr.Map, units, n_tiles: int = 12, rng_seed: i
             e = float(np.max(np.abs(lse_g[h, rows] - orc.lse[h, rows])))
             stats["lse_err"] = max(stats["lse_err"], e)
             assert e <= 1e-4, (h, I, e)
-    # stored probabilities of a sample of tiles kept by both sides
+    # stored probabilities: every tile kept by both sides (all_tiles), else a sample of them
     rng = np.random.default_rng(rng_seed)
     cand = []
     for u in units:
         h, I = divmod(u, nqb)
         for J in np.nonzero(kept_g[h, I, : I + 1] & orc.kept[h, I, : I + 1])[0]:
             cand.append((h, I, int(J)))
-    pick = [cand[i] for i in rng.choice(len(cand), size=min(n_tiles, len(cand)), replace=False)] if cand else []
-    # always include a diagonal tile and tile J = 0 when available
-    for extra in ((lambda c: c[1] == c[2]), (lambda c: c[2] == 0)):
-        sel = [c for c in cand if extra(c)]
-        if sel:
-            pick.append(sel[0])
+    if all_tiles:
+        pick = cand
+    else:
+        pick = [cand[i] for i in rng.choice(len(cand), size=min(n_tiles, len(cand)), replace=False)] if cand else []
+        # always include a diagonal tile and tile J = 0 when available
+        for extra in ((lambda c: c[1] == c[2]), (lambda c: c[2] == 0)):
+            sel = [c for c in cand if extra(c)]
+            if sel:
+                pick.append(sel[0])
     if pick:
         vals = m.export()
-        rtol, atol = VAL_TOL[spec.dtype]
-        vals_h = {}
+        vals_host = vals.cpu().numpy() if all_tiles else None  # reduced sizes: one host copy
+        col = m.col_idx.cpu().numpy()
+        rtol, atol = VAL_TOL[val_kind or spec.dtype]
+        by_unit = {}
         for (h, I, J) in pick:
-            u = h * nqb + I
-            bits = kept_g[h, I]
-            t = int(row_ptr[u] + bits[:J].sum())
-            if t >= m.capacity:
-                continue
-            got = vals[t].cpu().numpy().astype(np.float64)
-            want = oracle.tile_probs(lay.Q, lay.K, spec.scale, B, h, I, J, lay.bias)
-            err = np.abs(got - want)
-            assert np.all(err <= rtol * np.abs(want) + atol), (h, I, J, float(err.max()))
-            stats["val_err"] = max(stats["val_err"], float(np.max(err / (np.abs(want) + 1e-30) * (want > 1e-6))))
-            assert int(m.col_idx[t].item()) == J
+            by_unit.setdefault(h * nqb + I, []).append(J)
+        ulist = sorted(by_unit)
+        for c0 in range(0, len(ulist), 32):      # bounded memory: 32 row blocks of oracle rows at a time
+            chunk = ulist[c0:c0 + 32]
+            slab = oracle.row_block_probs(lay.Q, lay.K, spec.scale, B, chunk, lay.bias)
+            for k, u in enumerate(chunk):
+                h, I = divmod(u, nqb)
+                bits = kept_g[h, I]
+                for J in by_unit[u]:
+                    t = int(row_ptr[u] + bits[:J].sum())
+                    if t >= m.capacity:
+                        continue
+                    # full sizes: one tile at a time (the whole export would not fit in host memory)
+                    got = (vals_host[t] if all_tiles else vals[t].cpu().numpy()).astype(np.float64)
+                    want = slab[k][:, J * B:(J + 1) * B]
+                    err = np.abs(got - want)
+                    assert np.all(err <= rtol * np.abs(want) + atol), (h, I, J, float(err.max()))
+                    stats["val_err"] = max(stats["val_err"],
+                                           float(np.max(err / (np.abs(want) + 1e-30) * (want > 1e-6))))
+                    assert int(col[t]) == J
+                    stats["tiles_checked"] = stats.get("tiles_checked", 0) + 1
     return stats
 
 
-def compare_retrieve(spec, lay, m: mr.Map, O: torch.Tensor, rows, V=None, reqs=None):
+def compare_retrieve(spec, lay, m: mr.Map, O: torch.Tensor, rows, V=None, reqs=None, out_kind: str = None):
     """O [n_req][H_r][L][d_v] from the GPU vs the oracle on the GPU's own kept sets."""
     kept_g = m.kept_bits_host()
     V = lay.V if V is None else V
@@ -142,5 +163,5 @@ def compare_retrieve(spec, lay, m: mr.Map, O: torch.Tensor, rows, V=None, reqs=N
     got = O[:, :, rows].float().cpu().numpy() if reqs is None else O[reqs][:, :, rows].float().cpu().numpy()
     err = float(np.max(np.abs(got - want)))
     vmax = float(np.max(np.abs(V)))
-    assert err <= OUT_TOL[spec.dtype] * vmax, (err, vmax)
+    assert err <= OUT_TOL[out_kind or spec.dtype] * vmax, (err, vmax)
     return err / vmax

@@ -82,28 +82,46 @@ def test_compress_rejects_bad_arguments_without_launching(mr):
     bad_bias = mr.LogitBias(0, 0.0, 0, 0.0, fake, 0, 8)             # kb table without a block size
     assert lib.mr_compress(fake, fake, 0, 4, 512, 64, 0.125, 0.9, ctypes.byref(bad_bias), ctypes.byref(b),
                            fake, ws_bytes, None) == mr.MR_ERR_INVALID_ARG
+    # query-block range of mr_compress_blocks: 0 <= begin < end <= L / block (= 8 here)
+    blk = lambda q0, q1: lib.mr_compress_blocks(fake, fake, 0, 4, 512, 64, 0.125, 0.9, None, q0, q1,
+                                                ctypes.byref(b), fake, ws_bytes, None)
+    for q0, q1 in ((0, 0), (4, 4), (5, 3), (-1, 2), (0, 9)):
+        assert blk(q0, q1) == mr.MR_ERR_INVALID_ARG
 
 
 def test_retrieve_and_dense_reject_bad_arguments(mr):
     lib = mr.LIB
     fake = 0x1000
     b = _bsr(mr)
-    r = lambda **kw: lib.mr_retrieve(ctypes.byref(kw.get("b", b)), kw.get("W", fake), kw.get("H_r", 5), fake, fake,
-                                     kw.get("dt", 0), kw.get("dv", 64), kw.get("n", 1), None, 0,
-                                     kw.get("hs", 512 * 64), fake, 4096, None)
+    full = 5 * 512 * 64  # elements of [5][512][64] values
+
+    def r(**kw):
+        o = kw.get("opts")
+        return lib.mr_retrieve(ctypes.byref(kw.get("b", b)), kw.get("W", fake), kw.get("H_r", 5), fake,
+                               kw.get("ve", full), fake, kw.get("dt", 0), kw.get("dv", 64), kw.get("n", 1), None,
+                               kw.get("rs", 0), kw.get("hs", 512 * 64), ctypes.byref(o) if o else None, fake,
+                               kw.get("wsb", 4096 + 256), None)
     assert r(W=None) == mr.MR_ERR_INVALID_ARG
     assert r(dv=80) == mr.MR_ERR_UNSUPPORTED
     assert r(H_r=0) == mr.MR_ERR_INVALID_ARG
     assert r(n=0) == mr.MR_ERR_INVALID_ARG
     assert r(hs=10) == mr.MR_ERR_INVALID_ARG
     assert r(dt=1) == mr.MR_ERR_UNSUPPORTED
+    # the values must fit inside the stated allocation: heads x rows, and every request
+    assert r(ve=0) == mr.MR_ERR_INVALID_ARG
+    assert r(ve=full - 1) == mr.MR_ERR_INVALID_ARG
+    assert r(n=2, rs=full, ve=2 * full - 64) == mr.MR_ERR_INVALID_ARG
+    # options: query-block range inside the map, value groups dividing the receiver heads
+    assert r(opts=mr.RetrieveOpts(3, 3, 1)) == mr.MR_ERR_INVALID_ARG
+    assert r(opts=mr.RetrieveOpts(0, 9, 1)) == mr.MR_ERR_INVALID_ARG      # 512 / 64 = 8 query blocks
+    assert r(opts=mr.RetrieveOpts(-1, 4, 1)) == mr.MR_ERR_INVALID_ARG
+    assert r(opts=mr.RetrieveOpts(0, 0, 2)) == mr.MR_ERR_INVALID_ARG      # 5 heads, groups of 2
+    assert r(opts=mr.RetrieveOpts(0, 0, -1)) == mr.MR_ERR_INVALID_ARG
     # the workspace holds the status header and one progress counter per CTA (up to 1024)
     need = lib.mr_retrieve_workspace_bytes(ctypes.byref(b), 5, 64, 1)
     assert need == 256 + 1024 * 4
-    ok_args = lambda wsb: lib.mr_retrieve(ctypes.byref(b), fake, 5, fake, fake, 0, 64, 1, None, 0, 512 * 64,
-                                          fake, wsb, None)
-    assert ok_args(need - 1) == mr.MR_ERR_INVALID_ARG  # rejected before anything is launched
-    assert ok_args(256) == mr.MR_ERR_INVALID_ARG
+    assert r(wsb=need - 1) == mr.MR_ERR_INVALID_ARG  # rejected before anything is launched
+    assert r(wsb=256) == mr.MR_ERR_INVALID_ARG
     d = lambda **kw: lib.mr_dense_ref(fake, fake, fake, fake, kw.get("dt", 0), 4, kw.get("d", 64), 64,
                                       kw.get("cu", fake), fake, None, 2, 100, 100, 0.125, None, fake, 4096, None)
     assert d(cu=None) == mr.MR_ERR_INVALID_ARG

@@ -62,7 +62,7 @@ def test_reduced_configs_all_units(mr, name):
         m, O, st = run_layer(mr, spec, lay)
         assert st == mr.MR_OK
         nqb = spec.L // spec.block
-        stats = compare_compress(spec, lay, m, list(range(spec.H_s * nqb)))
+        stats = compare_compress(spec, lay, m, list(range(spec.H_s * nqb)), all_tiles=True)
         rel = compare_retrieve(spec, lay, m, O, np.arange(spec.L))
         print(name, stats, "out_err/max|V|", rel)
 
@@ -73,8 +73,39 @@ def test_tiny_lengths(mr, L, block):
     lay = draw_layers(spec)[0]
     m, O, st = run_layer(mr, spec, lay)
     assert st == mr.MR_OK
-    compare_compress(spec, lay, m, list(range(spec.H_s * (L // block))))
+    compare_compress(spec, lay, m, list(range(spec.H_s * (L // block))), all_tiles=True)
     compare_retrieve(spec, lay, m, O, np.arange(L))
+
+
+@pytest.mark.parametrize("dtype,d,block", [("bf16", 128, 64), ("bf16", 128, 128),   # tensor-core path
+                                           ("f32", 64, 64), ("bf16", 64, 128)])      # CUDA-core path
+def test_exact_ties_zero_query(mr, dtype, d, block):
+    """Q = 0 and no bias: A_ij = 1/(i+1), so every off-diagonal key block of a query block has
+    exactly the same mass (in the oracle's fp64 and in the kernels' fp32: the same values summed in
+    the same order), and the kept sets are decided by the tie-break alone (smaller J first).  They
+    must equal the oracle's bit for bit, with no boundary exemption, on both kernel paths."""
+    import math
+    import oracle
+    from cross_model_attention_mr_b200.workloads import round_to_bf16
+    H, L = 2, 1024
+    nqb = L // block
+    Q = np.zeros((H, L, d), np.float32)
+    K = round_to_bf16(np.random.default_rng(17).standard_normal((H, L, d), dtype=np.float32))
+    scale = 1.0 / math.sqrt(d)
+    for p in (0.3, 0.7, 0.9):
+        orc = oracle.compress(Q, K, scale, p32(p), block, None)
+        for I in range(nqb):  # precondition: the oracle's cumulative mass is far from p at the boundary
+            M = orc.mass[0, I, : I + 1]
+            cum = np.cumsum(np.sort(M)[::-1])
+            k = int(orc.count[0, I])
+            assert all(abs(cum[t] - p32(p)) > 1e-4 for t in (k - 2, k - 1) if 0 <= t < len(cum))
+        m = mr.compress(dev(Q, dtype), dev(K, dtype), p32(p), block, bias=None, scale=scale, store_mass=True)
+        assert m.ws.sync_status() == mr.MR_OK
+        kept = m.kept_bits_host()
+        assert np.array_equal(kept, orc.kept), (dtype, d, block, p)
+        mass = m.mass.cpu().numpy().reshape(H, nqb, nqb)
+        for I in range(2, nqb):  # the off-diagonal blocks are tied exactly in the kernel too
+            assert np.unique(mass[:, I, :I]).size == 1, (I, np.unique(mass[:, I, :I]))
 
 
 @pytest.mark.parametrize("p", [1.0, 0.05])
@@ -88,7 +119,7 @@ def test_extreme_thresholds(mr, p):
     if p >= 1:
         assert np.array_equal(kept, np.tril(np.ones((nqb, nqb), np.uint8))[None].repeat(3, 0))
         assert m.nnz_host() == mr.max_tiles(3, 512, 64)
-    compare_compress(spec, lay, m, list(range(spec.H_s * nqb)))
+    compare_compress(spec, lay, m, list(range(spec.H_s * nqb)), all_tiles=True)
     compare_retrieve(spec, lay, m, O, np.arange(spec.L))
 
 
@@ -264,3 +295,244 @@ def test_full_size_sampled(mr, n):
     rows = np.array([0, 5, spec.L // 2 + 17, spec.L - 1])
     rel = compare_retrieve(spec, lay, m, O, rows)
     print(spec.name, stats, rel)
+
+
+def test_full_size_config3_two_layers(mr):
+    """28 layers x L=8192, 32 -> 28 heads, block 64, per-layer key-block bias shared by the heads:
+    the first and the last layer at full size, sampled units and rows (the benchmark runs every
+    layer through the same calls)."""
+    spec = config(3)
+    for li, lay in zip((0, 27), draw_layers(spec, [0, 27])):
+        m, O, st = run_layer(mr, spec, lay)
+        assert st == mr.MR_OK
+        stats = compare_compress(spec, lay, m, _sample_units(spec, 4, 30 + li), n_tiles=6)
+        rows = np.array([0, 63, 64, 4097, spec.L - 1])
+        rel = compare_retrieve(spec, lay, m, O, rows)
+        print(spec.name, "layer", li, stats, rel)
+        del m, O
+        torch.cuda.empty_cache()
+
+
+def test_full_size_config5_prefix_and_16_requests(mr):
+    """Shared 4096-token prefix compressed once, retrieved for all 16 requests through one packed
+    value buffer (per-request offsets), and every request's dense suffix rows (512-2048 tokens,
+    ragged) over its prefix + suffix keys: the benchmark's calls at full size."""
+    import oracle
+    from cross_model_attention_mr_b200.workloads import Bias as SpecBias, Layer
+    spec = config(5)
+    b = draw_batch(spec)
+    P, R = spec.L, spec.n_req
+    suffixes = [r.suffix for r in b.requests]
+    cu_k = np.concatenate([[0], np.cumsum([P + s for s in suffixes])]).astype(np.int32)
+    cu_q = np.concatenate([[0], np.cumsum(suffixes)]).astype(np.int32)
+    m = mr.compress(dev(b.Qs, "bf16"), dev(b.Ks, "bf16"), p32(spec.p), spec.block,
+                    bias=mr.Bias.from_spec(b.bias), scale=spec.scale, store_mass=True, store_lse=True)
+    assert m.ws.sync_status() == mr.MR_OK
+    pl = Layer(Q=b.Qs, K=b.Ks, V=None, W=b.W, bias=b.bias)
+    compare_compress(spec, pl, m, _sample_units(spec, 6, 55), n_tiles=8)
+    Vp = dev(np.concatenate([r.V for r in b.requests], axis=1), "bf16")
+    off = torch.tensor(cu_k[:-1].astype(np.int64) * spec.d_v, dtype=torch.int64, device="cuda")
+    ws_r = mr.Workspace(mr.retrieve_workspace_bytes(m, spec.H_r, spec.d_v, R))
+    O = mr.retrieve(m, torch.from_numpy(b.W).cuda(), Vp, v_req_off=off, v_head_stride=int(cu_k[-1]) * spec.d_v,
+                    n_req=R, ws=ws_r)
+    torch.cuda.synchronize()
+    check_retrieve_status(mr, ws_r)
+    rows = np.array([0, 1000, 2047, P - 1])
+    for q in range(R):
+        lay = Layer(Q=b.Qs, K=b.Ks, V=np.ascontiguousarray(b.requests[q].V[:, :P]), W=b.W, bias=b.bias)
+        compare_retrieve(spec, lay, m, O[q:q + 1], rows)
+    # dense suffix rows of every request
+    bias_r = mr.Bias(b.bias.sink_len, b.bias.sink_bias, b.bias.window, b.bias.window_bias)
+    Kp = dev(np.concatenate([r.K for r in b.requests], axis=1), "bf16")
+    Qsuf = dev(np.concatenate([r.Q[:, P:] for r in b.requests], axis=1), "bf16")
+    Od = mr.dense_ref(Qsuf, Kp, Vp, torch.from_numpy(cu_q).cuda(), torch.from_numpy(cu_k).cuda(),
+                      torch.full((R,), P, dtype=torch.int32, device="cuda"), int(cu_q[-1]), int(cu_k[-1]),
+                      bias_r, spec.scale)
+    torch.cuda.synchronize()
+    sb = SpecBias(b.bias.sink_len, b.bias.sink_bias, b.bias.window, b.bias.window_bias)
+    for q, r in enumerate(b.requests):
+        srows = np.array([0, r.suffix // 2, r.suffix - 1])
+        want = oracle.dense_rows(r.Q[:, P:], r.K, r.V, spec.scale, srows, P, sb)
+        got = Od[:, cu_q[q] + srows].float().cpu().numpy()
+        assert np.max(np.abs(got - want)) <= OUT_TOL["bf16"] * float(np.abs(r.V).max()), q
+
+
+# ------------------------------------------------------------------------------------------------
+# Query-block ranges (chunked prefill / one rank's share of a sequence split across GPUs),
+# grouped value heads, and value offsets checked against the allocation.
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("n,kw,cuts", [(2, dict(L=1024, H_s=4, H_r=5), (0, 5, 11, 16)),        # block 64, odd cut
+                                       (4, dict(L=2048, H_s=3, H_r=4), (0, 9, 16)),            # block 128
+                                       (1, dict(L=512, H_s=4, H_r=4), (0, 3, 8))])             # fp32, CUDA cores
+def test_block_ranges_reassemble_the_full_call(mr, n, kw, cuts):
+    """Compressing and retrieving query-block ranges separately (as ranks of a split sequence would)
+    gives exactly the full call's kept sets, stored tiles and output rows."""
+    spec = shrink(config(n), **kw)
+    lay = draw_layers(spec)[0]
+    B, nqb = spec.block, spec.L // spec.block
+    Q, K = dev(lay.Q, spec.dtype), dev(lay.K, spec.dtype)
+    V, W = dev(lay.V, spec.dtype), torch.from_numpy(lay.W).cuda()
+    bias = mr.Bias.from_spec(lay.bias)
+    full = mr.compress(Q, K, p32(spec.p), B, bias=bias, scale=spec.scale)
+    O_full = mr.retrieve(full, W, V)
+    torch.cuda.synchronize()
+    kept_full = full.kept_bits_host()
+    rp_full = full.row_ptr.cpu().numpy()
+    vals_full = full.export().cpu()
+    O = torch.full_like(O_full, float("nan"))
+    for q0, q1 in zip(cuts[:-1], cuts[1:]):
+        part = mr.compress(Q, K, p32(spec.p), B, bias=bias, scale=spec.scale, blocks=(q0, q1))
+        ws_r = mr.Workspace(mr.retrieve_workspace_bytes(part, spec.H_r, spec.d_v, 1))
+        mr.retrieve(part, W, V, out=O, ws=ws_r, blocks=(q0, q1))
+        torch.cuda.synchronize()
+        assert part.ws.sync_status() == mr.MR_OK
+        check_retrieve_status(mr, ws_r)
+        kept = part.kept_bits_host()
+        assert np.array_equal(kept[:, q0:q1], kept_full[:, q0:q1])
+        assert not kept[:, :q0].any() and not kept[:, q1:].any()
+        rp = part.row_ptr.cpu().numpy()
+        vals = part.export().cpu()
+        for h in range(spec.H_s):
+            for I in range(q0, q1):
+                u = h * nqb + I
+                a, b = rp[u], rp[u + 1]
+                fa, fb = rp_full[u], rp_full[u + 1]
+                assert b - a == fb - fa
+                assert torch.equal(vals[a:b], vals_full[fa:fb])
+    assert torch.equal(O, O_full)  # every row written exactly once, identical to the full call
+
+
+def test_grouped_value_heads(mr):
+    """8 receiver heads reading 2 value heads (groups of 4): the same as expanding V per receiver."""
+    from cross_model_attention_mr_b200.workloads import Layer
+    spec = shrink(config(2), L=768, H_s=4, H_r=8)
+    lay = draw_layers(spec)[0]
+    V2 = np.ascontiguousarray(lay.V[:2])
+    Vx = np.repeat(V2, 4, axis=0)  # receiver head r reads value head r // 4
+    Q, K = dev(lay.Q, "bf16"), dev(lay.K, "bf16")
+    m = mr.compress(Q, K, p32(spec.p), spec.block, bias=mr.Bias.from_spec(lay.bias), scale=spec.scale)
+    ws_r = mr.Workspace(mr.retrieve_workspace_bytes(m, spec.H_r, spec.d_v, 1))
+    O = mr.retrieve(m, torch.from_numpy(lay.W).cuda(), dev(V2, "bf16"), ws=ws_r, v_group=4)
+    torch.cuda.synchronize()
+    check_retrieve_status(mr, ws_r)
+    lx = Layer(Q=lay.Q, K=lay.K, V=Vx, W=lay.W, bias=lay.bias)
+    compare_retrieve(spec, lx, m, O, np.array([0, 1, 63, 64, 400, 767]))
+
+
+@pytest.mark.parametrize("dtype,d_v", [("bf16", 128), ("f32", 64)])
+def test_value_offset_outside_allocation_reads_zeros(mr, dtype, d_v):
+    """A device offset table entry whose rows would leave the stated V allocation: that request reads
+    zeros and the status word says MR_ERR_DEVICE_CHECK; the other requests are unaffected."""
+    from cross_model_attention_mr_b200.workloads import Layer
+    spec = shrink(config(2 if dtype == "bf16" else 1), L=512, H_s=3, H_r=2, d_v=d_v)
+    lay = draw_layers(spec)[0]
+    m = mr.compress(dev(lay.Q, dtype), dev(lay.K, dtype), p32(spec.p), spec.block,
+                    bias=mr.Bias.from_spec(lay.bias), scale=spec.scale)
+    Vp = dev(np.concatenate([lay.V, lay.V], axis=1), dtype)  # [H_r][2L][d_v]: two requests packed
+    seq = spec.L * d_v
+    bad = 4 * seq                                              # starts at the end of the allocation
+    off = torch.tensor([0, bad], dtype=torch.int64, device="cuda")
+    ws_r = mr.Workspace(mr.retrieve_workspace_bytes(m, spec.H_r, d_v, 2))
+    O = mr.retrieve(m, torch.from_numpy(lay.W).cuda(), Vp, v_req_off=off, v_head_stride=2 * seq, n_req=2, ws=ws_r)
+    torch.cuda.synchronize()
+    assert ws_r.sync_status() == mr.MR_ERR_DEVICE_CHECK
+    assert float(O[1].float().abs().max()) == 0.0
+    compare_retrieve(spec, Layer(Q=lay.Q, K=lay.K, V=lay.V, W=lay.W, bias=lay.bias), m, O[0:1],
+                     np.array([0, 100, 511]))
+
+
+def test_dense_tensor_core_ragged_with_key_block_bias(mr):
+    """The tensor-core dense kernel (bf16, d = d_v = 128): an empty sequence, sequences shorter than
+    one 128-row tile and longer than several, query offsets, and sink + window + per-key-block bias."""
+    import oracle
+    from cross_model_attention_mr_b200.workloads import Bias as SpecBias, round_to_bf16
+    H, d = 3, 128
+    seqs = [(0, 64), (70, 200), (300, 700), (129, 129)]           # (query rows, key rows)
+    rng = np.random.default_rng(123)
+    std = 4.0 / np.sqrt(d)
+    Qs = [round_to_bf16(rng.standard_normal((H, lq, d), dtype=np.float32) * np.float32(std)) for lq, _ in seqs]
+    Ks = [round_to_bf16(rng.standard_normal((H, lk, d), dtype=np.float32) * np.float32(std)) for _, lk in seqs]
+    Vs = [round_to_bf16(rng.standard_normal((H, lk, d), dtype=np.float32)) for _, lk in seqs]
+    n_kb = 18                                                      # covers the 1093 packed keys
+    kb = np.full((H, n_kb), -np.inf, np.float32)
+    kb[:, [1, 4, 9]] = np.float32(2.5)
+    sb = SpecBias(sink_len=16, sink_bias=3.0, window=128, window_bias=3.0, kb_bias=kb, kb_block=64)
+    cu_q = np.concatenate([[0], np.cumsum([a for a, _ in seqs])]).astype(np.int32)
+    cu_k = np.concatenate([[0], np.cumsum([b for _, b in seqs])]).astype(np.int32)
+    offs = np.array([b - a for a, b in seqs], np.int32)
+    O = mr.dense_ref(dev(np.concatenate(Qs, axis=1), "bf16"), dev(np.concatenate(Ks, axis=1), "bf16"),
+                     dev(np.concatenate(Vs, axis=1), "bf16"), torch.from_numpy(cu_q).cuda(),
+                     torch.from_numpy(cu_k).cuda(), torch.from_numpy(offs).cuda(), int(cu_q[-1]), int(cu_k[-1]),
+                     mr.Bias.from_spec(sb), 1.0 / np.sqrt(d))
+    torch.cuda.synchronize()
+    Oh = O.float().cpu().numpy()
+    assert np.all(np.isfinite(Oh))
+    for s, (lq, lk) in enumerate(seqs):
+        if lq == 0:
+            continue
+        want = oracle.dense_rows(Qs[s], Ks[s], Vs[s], 1.0 / np.sqrt(d), np.arange(lq), int(offs[s]), sb)
+        err = np.max(np.abs(Oh[:, cu_q[s]:cu_q[s + 1]] - want))
+        assert err <= OUT_TOL["bf16"] * float(np.abs(Vs[s]).max()), (s, err)
+
+
+def test_dense_full_length_sampled(mr):
+    """One 32768-token sequence (the length of the headline workload) with its sink + window bias,
+    8 heads, sampled rows across the whole length."""
+    import oracle
+    spec = shrink(config(4), H_s=8, H_r=8)
+    lay = draw_layers(spec)[0]
+    cu = torch.tensor([0, spec.L], dtype=torch.int32, device="cuda")
+    from cross_model_attention_mr_b200.workloads import Bias as SpecBias
+    sb = SpecBias(lay.bias.sink_len, lay.bias.sink_bias, lay.bias.window, lay.bias.window_bias)
+    O = mr.dense_ref(dev(lay.Q, "bf16"), dev(lay.K, "bf16"), dev(lay.V, "bf16"), cu, cu, None, spec.L, spec.L,
+                     mr.Bias.from_spec(sb), spec.scale)
+    torch.cuda.synchronize()
+    rows = np.array([0, 1, 127, 128, 5000, 16383, 30001, spec.L - 1])
+    want = oracle.dense_rows(lay.Q, lay.K, lay.V, spec.scale, rows, 0, sb)
+    got = O[:, rows].float().cpu().numpy()
+    assert np.max(np.abs(got - want)) <= OUT_TOL["bf16"] * float(np.abs(lay.V).max())
+
+
+# ------------------------------------------------------------------------------------------------
+# fp8 (e4m3) maps with a scale per 32-row x 64-key piece (the compact representation of the map)
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("n,kw", [(2, dict(L=1024, H_s=6, H_r=5)), (4, dict(L=2048, H_s=3, H_r=6)),
+                                  (2, dict(L=512, H_s=3, H_r=4, d_v=64))])   # d_v 64: CUDA-core retrieval
+def test_fp8_maps_against_the_oracle(mr, n, kw):
+    spec = shrink(config(n), **kw)
+    lay = draw_layers(spec)[0]
+    Q, K = dev(lay.Q, "bf16"), dev(lay.K, "bf16")
+    bias = mr.Bias.from_spec(lay.bias)
+    m8 = mr.compress(Q, K, p32(spec.p), spec.block, bias=bias, scale=spec.scale, store_mass=True, store_lse=True,
+                     map_dtype=mr.MR_FP8_E4M3)
+    m16 = mr.compress(Q, K, p32(spec.p), spec.block, bias=bias, scale=spec.scale)
+    assert m8.ws.sync_status() == mr.MR_OK
+    assert np.array_equal(m8.kept_bits_host(), m16.kept_bits_host())     # the same selection
+    nqb = spec.L // spec.block
+    stats = compare_compress(spec, lay, m8, list(range(spec.H_s * nqb)), all_tiles=True, val_kind="fp8")
+    assert int(m8.vals.view(torch.uint8).max()) <= 0x7e                  # finite, non-negative e4m3 codes
+    W, V = torch.from_numpy(lay.W).cuda(), dev(lay.V, "bf16")
+    ws_r = mr.Workspace(mr.retrieve_workspace_bytes(m8, spec.H_r, spec.d_v, 1))
+    O8 = mr.retrieve(m8, W, V, ws=ws_r)
+    torch.cuda.synchronize()
+    check_retrieve_status(mr, ws_r)
+    rel = compare_retrieve(spec, lay, m8, O8, np.arange(0, spec.L, 3), out_kind="fp8")
+    O16 = mr.retrieve(m16, W, V)
+    diff = float((O8.float() - O16.float()).abs().max()) / float(np.abs(lay.V).max())
+    print(spec.name, stats, "fp8 out err/max|V|", rel, "fp8 vs bf16", diff)
+
+
+def test_fp8_full_size_headline_workload(mr):
+    """The L=32768, 32 -> 64 heads workload with an fp8 map: sampled units, tiles and rows."""
+    spec = config(4)
+    lay = draw_layers(spec)[0]
+    m = mr.compress(dev(lay.Q, "bf16"), dev(lay.K, "bf16"), p32(spec.p), spec.block, bias=mr.Bias.from_spec(lay.bias),
+                    scale=spec.scale, store_mass=True, store_lse=True, map_dtype=mr.MR_FP8_E4M3)
+    assert m.ws.sync_status() == mr.MR_OK
+    stats = compare_compress(spec, lay, m, _sample_units(spec, 4, 4), n_tiles=6, val_kind="fp8")
+    ws_r = mr.Workspace(mr.retrieve_workspace_bytes(m, spec.H_r, spec.d_v, 1))
+    O = mr.retrieve(m, torch.from_numpy(lay.W).cuda(), dev(lay.V, "bf16"), ws=ws_r)
+    torch.cuda.synchronize()
+    check_retrieve_status(mr, ws_r)
+    rel = compare_retrieve(spec, lay, m, O, np.array([0, 5, spec.L // 2 + 17, spec.L - 1]), out_kind="fp8")
+    print(spec.name, "fp8", stats, rel)

@@ -59,10 +59,12 @@ def test_noalloc_matches_workspace_entry_point_twice_in_a_row(mr):
         cap = mr.max_tiles(spec.H_s, spec.L, spec.block)
         out = mr.Map(spec.H_s, spec.L, spec.block, mr._dt(Q), cap, "cuda")
         assert _noalloc(mr, Q, K, spec, bias, out) == mr.MR_OK
+        assert mr.compress_noalloc_status() == mr.MR_OK   # the device-side status of that call
         _same_map(mr, spec, out, ref)
         # a second call into the same (already used) scratch gives the same map again
         out2 = mr.Map(spec.H_s, spec.L, spec.block, mr._dt(Q), cap, "cuda")
         assert _noalloc(mr, Q, K, spec, bias, out2) == mr.MR_OK
+        assert mr.compress_noalloc_status() == mr.MR_OK
         _same_map(mr, spec, out2, ref)
 
 
@@ -74,7 +76,23 @@ def test_noalloc_fp32_workload(mr):
     ref = mr.compress(Q, K, p32(spec.p), spec.block, bias=bias, scale=spec.scale)
     out = mr.Map(spec.H_s, spec.L, spec.block, mr.MR_F32, mr.max_tiles(spec.H_s, spec.L, spec.block), "cuda")
     assert _noalloc(mr, Q, K, spec, bias, out) == mr.MR_OK
+    assert mr.compress_noalloc_status() == mr.MR_OK
     _same_map(mr, spec, out, ref)
+
+
+def test_noalloc_status_reports_capacity_overflow(mr):
+    """The status word of the fixed scratch is readable: a map that outgrows its capacity reports
+    MR_ERR_CAPACITY there, and the next call that fits reports MR_OK again."""
+    spec = shrink(config(2), L=512, H_s=2, H_r=2)
+    lay = draw_layers(spec)[0]
+    Q, K = dev(lay.Q, spec.dtype), dev(lay.K, spec.dtype)
+    bias = mr.Bias.from_spec(lay.bias)
+    small = mr.Map(spec.H_s, spec.L, spec.block, mr.MR_BF16, 5, "cuda")
+    assert _noalloc(mr, Q, K, spec, bias, small) == mr.MR_OK
+    assert mr.compress_noalloc_status() == mr.MR_ERR_CAPACITY
+    big = mr.Map(spec.H_s, spec.L, spec.block, mr.MR_BF16, mr.max_tiles(spec.H_s, spec.L, spec.block), "cuda")
+    assert _noalloc(mr, Q, K, spec, bias, big) == mr.MR_OK
+    assert mr.compress_noalloc_status() == mr.MR_OK
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch(mr):
