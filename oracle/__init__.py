@@ -57,10 +57,10 @@ def _load():
         lib.or_tile_probs.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, f64,
                                       ctypes.c_int] + bias_args + [ctypes.c_int] * 3 + [P]
         lib.or_row_block_probs.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, f64,
-                                           ctypes.c_int] + bias_args + [P, ctypes.c_int, P, ctypes.c_int]
+                                           ctypes.c_int] + bias_args + [P, ctypes.c_int, P, P, ctypes.c_int]
         lib.or_retrieve_rows.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, f64,
                                          ctypes.c_int] + bias_args + [
-            P, P, ctypes.c_int, P, ctypes.c_int, i64, ctypes.c_int, P, ctypes.c_int, P,
+            P, P, ctypes.c_int, P, ctypes.c_int, i64, ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P,
             ctypes.c_int]
         lib.or_dense_rows.argtypes = [P, P, P] + [ctypes.c_int] * 5 + [i64, f64] + bias_args + [
             P, ctypes.c_int, P, ctypes.c_int]
@@ -137,22 +137,26 @@ def tile_probs(Q, K, sigma: float, B: int, h: int, I: int, J: int, bias=None) ->
 
 
 def row_block_probs(Q, K, sigma: float, B: int, units: Sequence[int], bias=None,
-                    n_threads: int = 0) -> np.ndarray:
-    """Softmax rows of whole query blocks: [len(units)][B][L] for units u = h*nQB + I (s2.1)."""
+                    n_threads: int = 0, renorm_kept=None) -> np.ndarray:
+    """Softmax rows of whole query blocks: [len(units)][B][L] for units u = h*nQB + I (s2.1).
+    ``renorm_kept`` ([H][nQB][nKB] 0/1): the renormalised variant, kept blocks only, rows summing to 1."""
     Q, K = _f32(Q), _f32(K)
     H, L, d = Q.shape
     u = np.ascontiguousarray(units, dtype=np.int32)
     out = np.zeros((u.shape[0], B, L), np.float64)
     ba, keep = _bias_args(bias)
+    kp = None if renorm_kept is None else np.ascontiguousarray(renorm_kept, dtype=np.uint8)
     rc = _load().or_row_block_probs(_ptr(Q), _ptr(K), H, L, d, float(sigma), int(B), *ba, _ptr(u),
-                                    int(u.shape[0]), _ptr(out), int(n_threads))
+                                    int(u.shape[0]), _ptr(kp), _ptr(out), int(n_threads))
     if rc:
         raise ValueError("oracle row_block_probs rejected its arguments")
     return out
 
 
-def retrieve_rows(Q, K, sigma: float, B: int, kept, W, V, rows, bias=None, n_threads: int = 0):
-    """O[q][r][t][:] for query rows ``rows`` (absolute positions), on the given kept sets.
+def retrieve_rows(Q, K, sigma: float, B: int, kept, W, V, rows, bias=None, n_threads: int = 0,
+                  renorm: bool = False):
+    """O[q][r][t][:] for query rows ``rows`` (absolute positions), on the given kept sets
+    (``renorm``: each sender head's kept row rescaled to sum to 1 first).
 
     V: [H_r][L][dv] or [n_req][H_r][L][dv]."""
     Q, K, W = _f32(Q), _f32(K), _f32(W)
@@ -168,7 +172,7 @@ def retrieve_rows(Q, K, sigma: float, B: int, kept, W, V, rows, bias=None, n_thr
     ba, keep = _bias_args(bias)
     rc = _load().or_retrieve_rows(_ptr(Q), _ptr(K), H_s, L, d, float(sigma), int(B), *ba,
                                   _ptr(kept), _ptr(W), H_r, _ptr(V), n_req, H_r * L * dv, dv,
-                                  _ptr(rows), int(rows.shape[0]), _ptr(O), int(n_threads))
+                                  _ptr(rows), int(rows.shape[0]), 1 if renorm else 0, _ptr(O), int(n_threads))
     if rc:
         raise ValueError("oracle retrieve rejected its arguments")
     return O

@@ -23,7 +23,8 @@
  *     sum_J M_IJ = 1;
  *   - selection: order J <= I by mass descending, ties to the smaller J; keep the first k blocks
  *     with k the least k >= 1 whose cumulative fp64 mass (in that order) is >= p; p >= 1 keeps all;
- *   - kept probabilities are stored as they are (no renormalisation);
+ *   - kept probabilities are stored as they are (no renormalisation); the renormalised variant
+ *     divides each head's kept row by its kept mass (or_row_block_probs / or_retrieve_rows flag);
  *   - translated map  At_r[i,j] = sum_s W[r,s] A_s[i,j] [block(j) kept for (s, block(i))];
  *     output O_r[i] = sum_{j <= i} At_r[i,j] V_r[j].
  */
@@ -100,6 +101,17 @@ static double row_probs(const float* q, const float* Kh, int d, int64_t n_keys, 
     }
     for (int64_t j = 0; j < n_keys; ++j) out[j] /= l;
     return m + log(l);
+}
+
+/* Renormalised top-p row (the variant where the kept probabilities of a row are rescaled to sum
+ * to 1; the pages leave renormalisation open): row[j] over keys j < n_keys of the row becomes
+ * row[j] / sum_{j in kept blocks} row[j] for kept blocks and 0 elsewhere.  kept_row: [nKB] 0/1. */
+static void renormalise_row(double* row, int64_t n_keys, const uint8_t* kept_row, int B)
+{
+    double m = 0.0;
+    for (int64_t j = 0; j < n_keys; ++j)
+        if (kept_row[j / B]) m += row[j];
+    for (int64_t j = 0; j < n_keys; ++j) row[j] = (kept_row[j / B] && m > 0.0) ? row[j] / m : 0.0;
 }
 
 static void fill_bias(or_bias* b, int32_t sink_len, double sink_bias, int32_t window,
@@ -243,7 +255,8 @@ OR_EXPORT int or_tile_probs(const float* Q, const float* K, int H, int L, int d,
 OR_EXPORT int or_row_block_probs(const float* Q, const float* K, int H, int L, int d, double sigma,
                                  int B, int32_t sink_len, double sink_bias, int32_t window,
                                  double window_bias, const float* kb_bias, int32_t kb_block,
-                                 const int32_t* units, int n_units, double* out, int n_threads)
+                                 const int32_t* units, int n_units, const uint8_t* kept, double* out,
+                                 int n_threads)
 {
     if (B <= 0 || L % B) return 1;
     const int nQB = L / B;
@@ -265,6 +278,7 @@ OR_EXPORT int or_row_block_probs(const float* Q, const float* K, int H, int L, i
         row_probs(Q + ((int64_t)h * L + i) * d, K + (int64_t)h * L * d, d, i + 1, sigma, &bias, h, i,
                   row);
         for (int64_t j = i + 1; j < L; ++j) row[j] = 0.0;
+        if (kept) renormalise_row(row, i + 1, kept + ((int64_t)h * nQB + I) * nQB, B);
     }
     return 0;
 }
@@ -284,7 +298,7 @@ OR_EXPORT int or_retrieve_rows(const float* Q, const float* K, int H_s, int L, i
                                double window_bias, const float* kb_bias, int32_t kb_block,
                                const uint8_t* kept, const float* W, int H_r, const float* V,
                                int n_req, int64_t v_req_stride, int dv, const int64_t* rows,
-                               int n_rows, double* O, int n_threads)
+                               int n_rows, int renorm, double* O, int n_threads)
 {
     if (B <= 0 || L % B) return 1;
     const int nQB = L / B, nKB = L / B;
@@ -309,8 +323,12 @@ OR_EXPORT int or_retrieve_rows(const float* Q, const float* K, int H_s, int L, i
                 row_probs(Q + ((int64_t)s * L + i) * d, K + (int64_t)s * L * d, d, i + 1, sigma,
                           &bias, s, i, a);
                 const uint8_t* ks = kept + ((int64_t)s * nQB + I) * nKB;
-                for (int64_t j = 0; j <= i; ++j)
-                    if (!ks[j / B]) a[j] = 0.0;
+                if (renorm) {
+                    renormalise_row(a, i + 1, ks, B);
+                } else {
+                    for (int64_t j = 0; j <= i; ++j)
+                        if (!ks[j / B]) a[j] = 0.0;
+                }
             }
             for (int r = 0; r < H_r; ++r) {
                 for (int64_t j = 0; j <= i; ++j) {

@@ -424,3 +424,47 @@ def test_row_block_probs_match_torch_softmax(oracle_mod, n, kw):
         J = I // 2
         tile = oracle_mod.tile_probs(lay.Q, lay.K, spec.scale, B, h, I, J, lay.bias)
         assert np.array_equal(got[t][:, J * B:(J + 1) * B], tile)
+
+
+# ---------------------------------------------------------------------------------------------
+# The renormalised variant (kept probabilities of each head's row rescaled to sum to 1): equal to
+# torch's float64 softmax over the biased logits with every unkept key masked out.
+# ---------------------------------------------------------------------------------------------
+def test_renormalised_rows_are_the_masked_softmax(oracle_mod):
+    spec = _small(2, L=512, H_s=3)
+    lay = draw_layers(spec)[0]
+    B, nqb = spec.block, spec.L // spec.block
+    r = oracle_mod.compress(lay.Q, lay.K, spec.scale, 0.8, B, lay.bias)
+    units = [0, nqb - 1, 1 * nqb + 5, 2 * nqb + 3]
+    got = oracle_mod.row_block_probs(lay.Q, lay.K, spec.scale, B, units, lay.bias, renorm_kept=r.kept)
+    logits = spec.scale * np.einsum("hid,hjd->hij", lay.Q.astype(np.float64), lay.K.astype(np.float64))
+    logits = logits + _mask_from_rule(spec.H_s, spec.L, spec.L, lay.bias)
+    for t, u in enumerate(units):
+        h, I = divmod(u, nqb)
+        keep_keys = np.repeat(r.kept[h, I], B).astype(bool)           # [L] kept keys of this row block
+        lg = np.where(keep_keys[None, :], logits[h, I * B:(I + 1) * B], -np.inf)
+        ref = torch.softmax(torch.from_numpy(lg), dim=-1).numpy()
+        assert np.max(np.abs(got[t] - ref)) < 1e-13
+        assert np.max(np.abs(got[t].sum(axis=1) - 1.0)) < 1e-12
+
+
+def test_renormalised_retrieval_matches_masked_softmax_mix(oracle_mod):
+    """O_r = (sum_s W[r,s] masked_softmax_s) V_r with torch; with every block kept it is the plain
+    retrieval."""
+    spec = _small(2, L=256, H_s=3, H_r=4)
+    lay = draw_layers(spec)[0]
+    B, nqb = spec.block, spec.L // spec.block
+    r = oracle_mod.compress(lay.Q, lay.K, spec.scale, 0.7, B, lay.bias)
+    rows = np.array([0, 70, 129, 255])
+    got = oracle_mod.retrieve_rows(lay.Q, lay.K, spec.scale, B, r.kept, lay.W, lay.V, rows, lay.bias, renorm=True)
+    logits = spec.scale * np.einsum("hid,hjd->hij", lay.Q.astype(np.float64), lay.K.astype(np.float64))
+    logits = logits + _mask_from_rule(spec.H_s, spec.L, spec.L, lay.bias)
+    keep = np.repeat(np.repeat(r.kept, B, axis=1), B, axis=2).astype(bool)   # [H][L][L]
+    A = torch.softmax(torch.from_numpy(np.where(keep, logits, -np.inf)), dim=-1).numpy()
+    At = np.einsum("rs,sij->rij", lay.W.astype(np.float64), A)
+    want = np.einsum("rij,rjc->ric", At[:, rows], lay.V.astype(np.float64))
+    assert np.max(np.abs(got[0] - want)) < 1e-12
+    allk = np.tril(np.ones((nqb, nqb), np.uint8))[None].repeat(spec.H_s, 0)
+    a = oracle_mod.retrieve_rows(lay.Q, lay.K, spec.scale, B, allk, lay.W, lay.V, rows, lay.bias, renorm=True)
+    b = oracle_mod.retrieve_rows(lay.Q, lay.K, spec.scale, B, allk, lay.W, lay.V, rows, lay.bias)
+    assert np.max(np.abs(a - b)) < 1e-13
