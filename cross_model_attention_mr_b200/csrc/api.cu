@@ -184,6 +184,16 @@ mr_status mr_retrieve(const mr_bsr* map, const float* W, int H_r, const void* V,
   if (fp8 && !map->tile_scale) return MR_ERR_INVALID_ARG;
   const int nqb = map->L / map->block;
   int qb0 = 0, qb1 = nqb, group = 1;
+  const int32_t* pages = nullptr;
+  int page_rows = 0, pages_per_req = 0;
+  if (opts && opts->v_pages) {
+    pages = opts->v_pages;
+    page_rows = opts->page_rows;
+    pages_per_req = opts->pages_per_req;
+    if (page_rows < 64 || page_rows % 64 || pages_per_req < 1 ||
+        (int64_t)pages_per_req * page_rows < map->L)
+      return MR_ERR_INVALID_ARG;
+  }
   if (opts) {
     if (opts->qb_begin != 0 || opts->qb_end != 0) {
       qb0 = opts->qb_begin;
@@ -196,9 +206,11 @@ mr_status mr_retrieve(const mr_bsr* map, const float* W, int H_r, const void* V,
   }
   const int H_v = H_r / group;
   const int64_t seq = (int64_t)map->L * d_v;
-  if (H_v > 1 && v_head_stride < seq) return MR_ERR_INVALID_ARG;
+  if (!(opts && opts->v_pages) && H_v > 1 && v_head_stride < seq) return MR_ERR_INVALID_ARG;
   // strided values: the furthest element read must lie inside the allocation
-  if (!v_req_off) {
+  if (pages) {
+    if ((int64_t)page_rows * d_v * H_v > v_elems) return MR_ERR_INVALID_ARG;  // not even one page fits
+  } else if (!v_req_off) {
     const int64_t last = (int64_t)(n_req - 1) * v_req_stride + (int64_t)(H_v - 1) * v_head_stride + seq;
     if (last > v_elems) return MR_ERR_INVALID_ARG;
   } else if (seq > v_elems) {
@@ -223,6 +235,9 @@ mr_status mr_retrieve(const mr_bsr* map, const float* W, int H_r, const void* V,
   a.v_group = group;
   a.qb0 = qb0;
   a.qb1 = qb1;
+  a.v_pages = pages;
+  a.page_rows = page_rows;
+  a.pages_per_req = pages_per_req;
   a.ws = (WsHeader*)ws;
   a.stream = st;
   return from_cuda(tc_retrieve_supported(a) ? tc_retrieve(a) : simt_retrieve(a));

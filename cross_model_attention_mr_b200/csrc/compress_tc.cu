@@ -47,6 +47,7 @@ struct Params {
   int H, L, B, nqb, nkw, n_rb, n_units;
   int rb_hi;     // units cover 128-row blocks rb_hi - n_rb .. rb_hi - 1
   int qb0, qb1;  // query blocks whose selection is written
+  int renorm;    // stored rows are divided by their kept mass (the emit's normaliser absorbs it)
   float a;  // logit scale in base 2: scale * log2(e)
   float p;
   Bias bias;
@@ -221,6 +222,11 @@ __device__ void softmax_group(Smem& s, const Params& p, int w) {
     float c = -INFINITY;                   // row reference (base 2)
     int used = 0;                          // block-sum columns written in this unit
     for (int T = w; T <= rb; T += 2) {
+      // the key-block bias terms of this tile (one per 32 keys), fetched before the wait for S so
+      // their latency hides behind the MMA
+      float kbo[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) kbo[c] = kb_offset(p.bias, h, 128 * T + 32 * c);
       if (!mbar_wait(&s.s_full[w], nb & 1, &s.abort, kTimeoutNs)) {
         // Leave the tile loop but still pass the epilogue's barriers of this unit: the other
         // warpgroup's bounded waits see the abort flag and meet us there.
@@ -259,8 +265,8 @@ __device__ void softmax_group(Smem& s, const Params& p, int w) {
         float mc;
         if (!special) {
           // only the key-block term can apply: a constant per 32 keys
-          off[0] = kb_offset(p.bias, h, j0);
-          off[1] = kb_offset(p.bias, h, j0 + 32);
+          off[0] = kbo[2 * hh];
+          off[1] = kbo[2 * hh + 1];
           mc = fmaxf(fmaf(warp_max32(v[0]), p.a, off[0]), fmaf(warp_max32(v[1]), p.a, off[1]));
         } else {
 #pragma unroll
@@ -453,6 +459,30 @@ __device__ void softmax_group(Smem& s, const Params& p, int w) {
         for (int J = gtid; J < p.nqb; J += 128) p.mass_out[(size_t)u * p.nqb + J] = J <= I ? m[J] : 0.f;
     }
     named_sync(1, 256);  // the shared arrays are reused by the next unit
+    if (p.renorm) {
+      // kept mass of this thread's row: its normalised block sums of the kept blocks of the row's
+      // query block, over both warpgroups' columns; the emit's normaliser then absorbs it
+      const int qrow = (p.B == 128) ? 0 : (row >> 6);
+      const int Irow = (p.B == 128) ? rb : 2 * rb + qrow;
+      float part = 0.f;
+      for (int c0 = 0; c0 < used; c0 += 32) {
+        uint32_t xs[32];
+        tmem_ld32(tbase + lane_addr + xbase + c0, xs);
+        tmem_wait_ld();
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          const int col = c0 + t;
+          const int J = (p.B == 128) ? 2 * col + w : 4 * (col >> 1) + 2 * w + (col & 1);
+          if (col < used && J <= Irow && ((s.bits[qrow][J >> 5] >> (J & 31)) & 1u)) part += __uint_as_float(xs[t]);
+        }
+      }
+      s.csum[w][row] = part * scale;
+      named_sync(1, 256);
+      if (w == 0 && row_ok && good && Irow >= p.qb0 && Irow < p.qb1) {
+        const float m = s.csum[0][row] + s.csum[1][row];
+        if (m > 0.f) p.lse_ws[(size_t)h * p.L + i] += logf(m);
+      }
+    }
     const bool stop = s.sm_fail != 0;
     named_sync(1, 256);  // nobody starts the next unit's tiles before everyone has read the flag
     if (stop) break;
@@ -521,6 +551,7 @@ cudaError_t tc_compress_stats(const CompressArgs& a) {
   p.n_units = p.H * p.n_rb;
   p.qb0 = a.qb0;
   p.qb1 = a.qb1;
+  p.renorm = a.map.renormalised != 0;
   p.a = a.scale * kLog2e;
   p.p = a.p;
   p.bias = a.bias;

@@ -36,6 +36,8 @@ struct RetrieveArgs {
   int64_t v_req_stride, v_head_stride;
   int v_group;      // receiver heads per value head
   int qb0, qb1;     // output query blocks: qb0 <= I < qb1
+  const int32_t* v_pages;  // paged values: [n_req][pages_per_req] page numbers, or nullptr
+  int page_rows, pages_per_req;
   WsHeader* ws;
   cudaStream_t stream;
 };

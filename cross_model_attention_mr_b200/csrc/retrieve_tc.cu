@@ -69,6 +69,9 @@ struct Params {
   int64_t v_req_stride, v_head_stride;
   int64_t v_rows;  // rows of 128 values in the V allocation (the tensor map's extent)
   int v_group;     // receiver heads per value head
+  int H_v;         // value heads
+  const int32_t* v_pages;  // paged values: [n_req][pages_per_req] page numbers, or nullptr
+  int page_rows, pages_per_req;
   int H_s, H_r, L, B, nqb, nkw, n_req;
   int R, n_hg, n_rg, n_rb, n_units;
   int rb_hi;       // 128-row blocks rb_hi - n_rb .. rb_hi - 1 hold the output query blocks
@@ -413,14 +416,25 @@ __device__ void issue_v(S& s, const Params& p, const CUtensorMap* tmap_v, const 
   for (int a = 0; a < G * p.R; ++a) {
     if (!acc_valid(p, u, G, a)) continue;
     const int r = u.hg * G + a / p.R, q = u.rg * p.R + a % p.R;
-    const int64_t off = (p.v_req_off ? p.v_req_off[q] : (int64_t)q * p.v_req_stride) +
-                        (int64_t)(r / p.v_group) * p.v_head_stride;
-    // a request's rows must start on a row of the tensor map and end inside the allocation; if
-    // not, load from past the map's extent (TMA fills zeros) and record the bad offset
-    int64_t row = off / 128 + j0;
-    if (off < 0 || (off & 127) != 0 || off / 128 + (int64_t)p.L > p.v_rows) {
-      set_status(p.ws, MR_ERR_DEVICE_CHECK, 5u);
-      row = p.v_rows;
+    const int g = r / p.v_group;
+    int64_t row;
+    if (p.v_pages) {
+      // paged values: the 64 rows j0 .. j0 + 63 lie in one page (page_rows is a multiple of 64)
+      const int64_t page = p.v_pages[(int64_t)q * p.pages_per_req + j0 / p.page_rows];
+      row = (page * p.H_v + g) * p.page_rows + j0 % p.page_rows;
+      if (page < 0 || (page * p.H_v + g + 1) * p.page_rows > p.v_rows) {
+        set_status(p.ws, MR_ERR_DEVICE_CHECK, 6u);
+        row = p.v_rows;
+      }
+    } else {
+      const int64_t off = (p.v_req_off ? p.v_req_off[q] : (int64_t)q * p.v_req_stride) + (int64_t)g * p.v_head_stride;
+      // a request's rows must start on a row of the tensor map and end inside the allocation; if
+      // not, load from past the map's extent (TMA fills zeros) and record the bad offset
+      row = off / 128 + j0;
+      if (off < 0 || (off & 127) != 0 || off / 128 + (int64_t)p.L > p.v_rows) {
+        set_status(p.ws, MR_ERR_DEVICE_CHECK, 5u);
+        row = p.v_rows;
+      }
     }
     tma_load_2d(&s.v[a][0], tmap_v, &s.v_full, 0, (int)row);
     tma_load_2d(&s.v[a][64 * 64], tmap_v, &s.v_full, 64, (int)row);
@@ -915,8 +929,9 @@ cudaError_t launch_any(const RetrieveArgs& a, const Params& p, const CUtensorMap
 
 bool tc_retrieve_supported(const RetrieveArgs& a) {
   return a.dt == MR_BF16 && (a.map.val_dtype == MR_BF16 || a.map.val_dtype == MR_FP8_E4M3) && a.d_v == 128 && (a.map.block == 64 || a.map.block == 128) && a.map.H_s <= 64 &&
-         a.map.capacity_tiles < (int64_t)kNone && a.v_head_stride % 128 == 0 &&
-         (a.v_req_off != nullptr || a.v_req_stride % 128 == 0) && a.v_elems / 128 < ((int64_t)1 << 31) - 1;
+         a.map.capacity_tiles < (int64_t)kNone && (a.v_pages != nullptr || a.v_head_stride % 128 == 0) &&
+         (a.v_pages != nullptr || a.v_req_off != nullptr || a.v_req_stride % 128 == 0) &&
+         a.v_elems / 128 < ((int64_t)1 << 31) - 1;
 }
 
 cudaError_t tc_retrieve(const RetrieveArgs& a) {
@@ -934,6 +949,10 @@ cudaError_t tc_retrieve(const RetrieveArgs& a) {
   p.v_head_stride = a.v_head_stride;
   p.v_rows = a.v_elems / 128;
   p.v_group = a.v_group;
+  p.H_v = a.H_r / a.v_group;
+  p.v_pages = a.v_pages;
+  p.page_rows = a.page_rows;
+  p.pages_per_req = a.pages_per_req;
   p.H_s = a.map.H_s;
   p.H_r = a.H_r;
   p.L = a.map.L;

@@ -74,7 +74,8 @@ template <typename T, int BLK, int D>
 __global__ void __launch_bounds__(kThreads) k_compress_stats(
     const T* __restrict__ Q, const T* __restrict__ K, int H, int L, float scale, float p, Bias bias,
     float* __restrict__ lse_ws, int* __restrict__ count_ws, uint32_t* __restrict__ kept_bits,
-    float* __restrict__ kept_mass, float* __restrict__ mass_out, float* __restrict__ lse_out, int qb_hi) {
+    float* __restrict__ kept_mass, float* __restrict__ mass_out, float* __restrict__ lse_out, int qb_hi,
+    int renorm) {
   extern __shared__ float smem[];
   float* Qs = smem;
   float* Ks = Qs + BLK * (D + 1);
@@ -195,6 +196,34 @@ __global__ void __launch_bounds__(kThreads) k_compress_stats(
   if (tid < nkw) kept_bits[(size_t)u * nkw + tid] = bits_s[tid];
   if (mass_out)
     for (int J = tid; J < nkb; J += kThreads) mass_out[(size_t)u * nkb + J] = (J <= I) ? mass_s[J] : 0.f;
+  if (!renorm) return;
+  // renormalised map: each row's kept mass, sum over kept blocks of exp(s - lse), is absorbed into
+  // the normaliser the emit pass divides by
+  for (int r = tid; r < BLK; r += kThreads) row_l[r] = 0.f;
+  for (int J = 0; J <= I; ++J) {
+    if (!((bits_s[J >> 5] >> (J & 31)) & 1u)) continue;
+    __syncthreads();
+    load_rows<T, BLK, D>(Ks, K + ((size_t)h * L + (size_t)J * BLK) * D, BLK);
+    __syncthreads();
+    float S[R][R];
+    tile_dot<BLK, BLK, D>(Qs, Ks, S);
+#pragma unroll
+    for (int a = 0; a < R; ++a) {
+      const int r = ty + 16 * a;
+      const int i = I * BLK + r;
+      float acc = 0.f;
+#pragma unroll
+      for (int b = 0; b < R; ++b) {
+        const int j = J * BLK + tx + 16 * b;
+        if (j <= i) acc += expf(S[a][b] * scale + bias_term(bias, h, i, j) - row_m[r]);
+      }
+      acc = group16_sum(acc);
+      if (tx == 0) row_l[r] += acc;
+    }
+  }
+  __syncthreads();
+  for (int r = tid; r < BLK; r += kThreads)
+    if (row_l[r] > 0.f) lse_ws[(size_t)h * L + (size_t)I * BLK + r] += logf(row_l[r]);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -283,7 +312,7 @@ __global__ void __launch_bounds__(kThreads) k_retrieve(
     MapVals<TM> mv, int64_t capacity, int H_s, int L, const float* __restrict__ W,
     int H_r, const T* __restrict__ V, int64_t v_elems, T* __restrict__ O,
     const int64_t* __restrict__ v_req_off, int64_t v_req_stride, int64_t v_head_stride, int v_group,
-    int qb_hi, WsHeader* ws) {
+    int qb_hi, const int32_t* __restrict__ v_pages, int page_rows, int pages_per_req, WsHeader* ws) {
   extern __shared__ float smem[];
   float* Xs = smem;                   // [BLK][BLK + 1]
   float* Vs = Xs + BLK * (BLK + 1);   // [BLK][DV + 1]
@@ -295,12 +324,27 @@ __global__ void __launch_bounds__(kThreads) k_retrieve(
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   constexpr int R = BLK / 16, C = DV / 16, E = BLK * BLK / kThreads;
   for (int s = tid; s < H_s; s += kThreads) Ws[s] = W[(size_t)r * H_s + s];
-  // value head r / v_group of request q; rows 0 .. (I + 1) * BLK - 1 must lie inside the allocation,
-  // else the request reads zeros and the status word records the bad offset
-  const int64_t voff = (v_req_off ? v_req_off[q] : (int64_t)q * v_req_stride) + (int64_t)(r / v_group) * v_head_stride;
-  const bool v_ok = voff >= 0 && voff + (int64_t)(I + 1) * BLK * DV <= v_elems;
+  // value head g = r / v_group of request q; rows 0 .. (I + 1) * BLK - 1 must lie inside the
+  // allocation, else the request reads zeros and the status word records the bad offset
+  const int g = r / v_group, H_v = H_r / v_group;
+  const int64_t voff = v_pages ? 0 : (v_req_off ? v_req_off[q] : (int64_t)q * v_req_stride) + (int64_t)g * v_head_stride;
+  bool v_ok = true;
+  if (v_pages) {
+    for (int pg = 0; pg <= ((I + 1) * BLK - 1) / page_rows; ++pg) {
+      const int64_t page = v_pages[(int64_t)q * pages_per_req + pg];
+      v_ok = v_ok && page >= 0 && (page * H_v + g + 1) * page_rows * DV <= v_elems;
+    }
+  } else {
+    v_ok = voff >= 0 && voff + (int64_t)(I + 1) * BLK * DV <= v_elems;
+  }
   if (!v_ok && tid == 0) set_status(ws, MR_ERR_DEVICE_CHECK, 4u);
   const T* Vr = V + (v_ok ? voff : 0);
+  // element offset of value row j (paged: row j % page_rows of the request's page j / page_rows)
+  auto vrow = [&](int j) -> const T* {
+    if (!v_pages) return Vr + (int64_t)j * DV;
+    const int64_t page = v_pages[(int64_t)q * pages_per_req + j / page_rows];
+    return V + ((page * H_v + g) * page_rows + j % page_rows) * DV;
+  };
   float acc[R][C];
 #pragma unroll
   for (int a = 0; a < R; ++a)
@@ -334,7 +378,10 @@ __global__ void __launch_bounds__(kThreads) k_retrieve(
       mv.coords(tid + e * kThreads, BLK, ra, cb);
       Xs[ra * (BLK + 1) + cb] = x[e];
     }
-    load_rows<T, BLK, DV>(Vs, Vr + (size_t)J * BLK * DV, BLK);
+    for (int e = tid; e < BLK * DV; e += kThreads) {
+      const int rr = e / DV, c = e - (e / DV) * DV;
+      Vs[rr * (DV + 1) + c] = to_f32(vrow(J * BLK + rr)[c]);
+    }
     __syncthreads();
 #pragma unroll 4
     for (int j = 0; j < BLK; ++j) {
@@ -545,7 +592,7 @@ cudaError_t compress_impl(const CompressArgs& a) {
     ProfScope ps(kKCompressStats, a.stream);
     k1<<<a.H * (a.qb1 - a.qb0), kThreads, smem, a.stream>>>(
         (const T*)a.Q, (const T*)a.K, a.H, a.L, a.scale, a.p, a.bias, a.lse_ws, a.count_ws,
-        a.map.kept_bits, a.map.kept_mass, a.map.mass, a.map.lse, a.qb1);
+        a.map.kept_bits, a.map.kept_mass, a.map.mass, a.map.lse, a.qb1, a.map.renormalised);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = launch_scan_counts(a.count_ws, a.H * nqb, a.map, a.ws, a.stream)) != cudaSuccess) return e;
@@ -584,7 +631,8 @@ cudaError_t retrieve_impl(const RetrieveArgs& a) {
   ProfScope ps(kKRetrieve, a.stream);
   k<<<grid, kThreads, smem, a.stream>>>(a.map.row_ptr, a.map.kept_bits, mv, a.map.capacity_tiles, a.map.H_s, a.map.L, a.W, a.H_r,
                                          (const T*)a.V, a.v_elems, (T*)a.O, a.v_req_off, a.v_req_stride,
-                                         a.v_head_stride, a.v_group, a.qb1, a.ws);
+                                         a.v_head_stride, a.v_group, a.qb1, a.v_pages, a.page_rows,
+                                         a.pages_per_req, a.ws);
   return cudaGetLastError();
 }
 

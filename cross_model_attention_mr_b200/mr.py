@@ -31,14 +31,15 @@ class LogitBias(ctypes.Structure):
 
 
 class RetrieveOpts(ctypes.Structure):
-    _fields_ = [("qb_begin", _c_i32), ("qb_end", _c_i32), ("v_group", _c_i32)]
+    _fields_ = [("qb_begin", _c_i32), ("qb_end", _c_i32), ("v_group", _c_i32), ("v_pages", _c_p),
+                ("page_rows", _c_i32), ("pages_per_req", _c_i32)]
 
 
 class BSR(ctypes.Structure):
     _fields_ = [("H_s", _c_i32), ("L", _c_i32), ("block", _c_i32), ("val_dtype", ctypes.c_int),
                 ("capacity_tiles", _c_i64), ("row_ptr", _c_p), ("col_idx", _c_p), ("vals", _c_p),
                 ("kept_mass", _c_p), ("kept_bits", _c_p), ("mass", _c_p), ("lse", _c_p), ("nnz", _c_p),
-                ("tile_scale", _c_p)]
+                ("tile_scale", _c_p), ("renormalised", _c_i32)]
 
 
 EXPORTS = {
@@ -178,7 +179,7 @@ class Map:
     """A compressed map: caller-owned device arrays described by an ``mr_bsr``."""
 
     def __init__(self, H_s: int, L: int, block: int, dtype: int, capacity: int, device="cuda",
-                 store_mass: bool = False, store_lse: bool = False):
+                 store_mass: bool = False, store_lse: bool = False, renormalised: bool = False):
         self.H_s, self.L, self.block, self.dtype, self.capacity = H_s, L, block, dtype, int(capacity)
         self.nqb = L // block
         self.nkw = (self.nqb + 31) // 32
@@ -198,7 +199,8 @@ class Map:
                      self.vals.data_ptr(), self.kept_mass.data_ptr(), self.kept_bits.data_ptr(),
                      self.mass.data_ptr() if self.mass is not None else None,
                      self.lse.data_ptr() if self.lse is not None else None, self.nnz.data_ptr(),
-                     self.tile_scale.data_ptr() if self.tile_scale is not None else None)
+                     self.tile_scale.data_ptr() if self.tile_scale is not None else None,
+                     1 if renormalised else 0)
 
     def nnz_host(self, stream=None) -> int:
         v = _c_i64(0)
@@ -324,10 +326,12 @@ def compress_workspace_bytes(H_s, L, d, block) -> int:
 def compress(Q: torch.Tensor, K: torch.Tensor, p: float, block: int, bias: Optional[Bias] = None,
              scale: Optional[float] = None, capacity: Optional[int] = None, out: Optional[Map] = None,
              ws: Optional[Workspace] = None, store_mass=False, store_lse=False, stream=None,
-             blocks: Optional[tuple] = None, map_dtype: Optional[int] = None) -> Map:
+             blocks: Optional[tuple] = None, map_dtype: Optional[int] = None,
+             renormalised: bool = False) -> Map:
     """mr_compress: Q, K [H_s][L][d] (bf16 or fp32, CUDA) -> Map.  ``blocks=(qb_begin, qb_end)``
     calls mr_compress_blocks: only those query blocks, the other rows of the map left empty.
-    ``map_dtype=MR_FP8_E4M3`` stores e4m3 values with per-piece scales (bf16 inputs)."""
+    ``map_dtype=MR_FP8_E4M3`` stores e4m3 values with per-piece scales (bf16 inputs);
+    ``renormalised=True`` stores each row divided by its kept mass."""
     _need_cuda(Q, K)
     H, L, d = Q.shape
     dt = _dt(Q)
@@ -335,7 +339,8 @@ def compress(Q: torch.Tensor, K: torch.Tensor, p: float, block: int, bias: Optio
         scale = 1.0 / math.sqrt(d)
     if out is None:
         cap = max_tiles(H, L, block) if capacity is None else capacity
-        out = Map(H, L, block, dt if map_dtype is None else map_dtype, cap, Q.device, store_mass, store_lse)
+        out = Map(H, L, block, dt if map_dtype is None else map_dtype, cap, Q.device, store_mass, store_lse,
+                  renormalised)
     if ws is None:
         ws = Workspace(compress_workspace_bytes(H, L, d, block), Q.device)
     out.ws = ws
@@ -357,12 +362,14 @@ def retrieve(m: Map, W: torch.Tensor, V: torch.Tensor, out: Optional[torch.Tenso
              v_req_off: Optional[torch.Tensor] = None, v_req_stride: Optional[int] = None,
              v_head_stride: Optional[int] = None, n_req: Optional[int] = None,
              ws: Optional[Workspace] = None, stream=None, blocks: Optional[tuple] = None,
-             v_group: int = 1, v_elems: Optional[int] = None) -> torch.Tensor:
+             v_group: int = 1, v_elems: Optional[int] = None, v_pages: Optional[torch.Tensor] = None,
+             page_rows: int = 0) -> torch.Tensor:
     """mr_retrieve: W [H_r][H_s] fp32; V [H_v][L][d_v] or [n_req][H_v][L][d_v] (or a packed buffer
     with explicit strides/offsets), H_v = H_r / v_group -> O [n_req][H_r][L][d_v].
     ``blocks=(qb_begin, qb_end)`` writes only those query blocks' rows of O; ``v_elems`` defaults to
-    the number of elements of V."""
-    _need_cuda(W, V, v_req_off)
+    the number of elements of V.  ``v_pages`` [n_req][pages_per_req] (int32, device) reads V as a
+    pool of pages [page][H_v][page_rows][d_v]."""
+    _need_cuda(W, V, v_req_off, v_pages)
     H_r = W.shape[0]
     dt = _dt(V)
     d_v = V.shape[-1]
@@ -380,9 +387,11 @@ def retrieve(m: Map, W: torch.Tensor, V: torch.Tensor, out: Optional[torch.Tenso
     if ws is None:
         ws = Workspace(retrieve_workspace_bytes(m, H_r, d_v, n_req), V.device)
     opts = None
-    if blocks is not None or v_group != 1:
+    if blocks is not None or v_group != 1 or v_pages is not None:
         b = blocks if blocks is not None else (0, 0)
-        opts = ctypes.byref(RetrieveOpts(int(b[0]), int(b[1]), int(v_group)))
+        opts = ctypes.byref(RetrieveOpts(int(b[0]), int(b[1]), int(v_group),
+                                         v_pages.data_ptr() if v_pages is not None else None, int(page_rows),
+                                         int(v_pages.shape[1]) if v_pages is not None else 0))
     check(LIB.mr_retrieve(ctypes.byref(m.c), W.data_ptr(), H_r, V.data_ptr(), int(v_elems), out.data_ptr(), dt,
                           d_v, n_req, v_req_off.data_ptr() if v_req_off is not None else None, int(v_req_stride),
                           int(v_head_stride), opts, ws.ptr, ws.nbytes, _stream(stream)), "mr_retrieve")

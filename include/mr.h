@@ -104,6 +104,11 @@ typedef struct {
  *   nnz       int64  [1]              number of kept tiles (may exceed capacity_tiles)
  *   tile_scale float [capacity_tiles][S]  MR_FP8_E4M3 maps only (else unused, may be NULL): the
  *             scale of each 32-row x 64-key piece, max(piece) / 448 (448 = largest e4m3 value)
+ *   renormalised  set by the caller before mr_compress: 0 stores the kept probabilities as they
+ *             are (each row of the map then sums to its kept mass, at most 1); 1 stores every row
+ *             divided by its kept mass, so a head's kept probabilities of each query sum to 1 (the
+ *             renormalised top-p map; the pages leave renormalisation open).  Masses, selection and
+ *             lse are the same either way.
  */
 typedef struct {
   int32_t H_s;
@@ -120,6 +125,7 @@ typedef struct {
   float* lse;
   int64_t* nnz;
   float* tile_scale;
+  int32_t renormalised;
 } mr_bsr;
 
 /* Library version (major * 100 + minor). */
@@ -243,11 +249,23 @@ size_t mr_retrieve_workspace_bytes(const mr_bsr* map, int H_r, int d_v, int n_re
  *   v_group           receiver heads that share one value head (grouped-query attention): receiver
  *                     head r reads value head r / v_group.  0 or 1: one value head per receiver
  *                     head.  H_r must be a multiple of v_group.
+ *   v_pages           paged values (MapFlow section 6, "PagedAttention"), or NULL: device int32
+ *                     [n_req][pages_per_req] page numbers.  Token j of request q is row
+ *                     j % page_rows of page v_pages[q * pages_per_req + j / page_rows], and V is a
+ *                     pool of pages laid out [page][H_v][page_rows][d_v] (H_v = H_r / v_group), so
+ *                     element (q, g, j, c) is at
+ *                     V + ((page * H_v + g) * page_rows + j % page_rows) * d_v + c.
+ *                     v_req_off, v_req_stride and v_head_stride are then ignored.  page_rows: a
+ *                     positive multiple of 64; pages_per_req * page_rows >= L.  A page number whose
+ *                     rows fall outside [0, v_elems) reads zeros and records MR_ERR_DEVICE_CHECK.
  */
 typedef struct {
   int32_t qb_begin;
   int32_t qb_end;
   int32_t v_group;
+  const int32_t* v_pages;
+  int32_t page_rows;
+  int32_t pages_per_req;
 } mr_retrieve_opts;
 
 /*

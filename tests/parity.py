@@ -75,7 +75,7 @@ def check_selection(M: np.ndarray, kept_o: np.ndarray, kept_g: np.ndarray, p: fl
 
 
 def compare_compress(spec, lay, m: mr.Map, units, n_tiles: int = 12, rng_seed: int = 0,
-                     all_tiles: bool = False, val_kind: str = None):
+                     all_tiles: bool = False, val_kind: str = None, renorm: bool = False):
     """Check masses, selection, row normalisers and stored values of the given units (h*nqb + I)
     against the oracle: every tile both sides kept when ``all_tiles``, else ``n_tiles`` sampled ones
     (plus a diagonal tile and a J = 0 tile).  Returns a dict of statistics."""
@@ -135,7 +135,9 @@ def compare_compress(spec, lay, m: mr.Map, units, n_tiles: int = 12, rng_seed: i
         ulist = sorted(by_unit)
         for c0 in range(0, len(ulist), 32):      # bounded memory: 32 row blocks of oracle rows at a time
             chunk = ulist[c0:c0 + 32]
-            slab = oracle.row_block_probs(lay.Q, lay.K, spec.scale, B, chunk, lay.bias)
+            # a renormalised map divides each row by its kept mass over the GPU's own kept set
+            slab = oracle.row_block_probs(lay.Q, lay.K, spec.scale, B, chunk, lay.bias,
+                                          renorm_kept=kept_g if renorm else None)
             for k, u in enumerate(chunk):
                 h, I = divmod(u, nqb)
                 bits = kept_g[h, I]
@@ -155,11 +157,13 @@ def compare_compress(spec, lay, m: mr.Map, units, n_tiles: int = 12, rng_seed: i
     return stats
 
 
-def compare_retrieve(spec, lay, m: mr.Map, O: torch.Tensor, rows, V=None, reqs=None, out_kind: str = None):
+def compare_retrieve(spec, lay, m: mr.Map, O: torch.Tensor, rows, V=None, reqs=None, out_kind: str = None,
+                     renorm: bool = False):
     """O [n_req][H_r][L][d_v] from the GPU vs the oracle on the GPU's own kept sets."""
     kept_g = m.kept_bits_host()
     V = lay.V if V is None else V
-    want = oracle.retrieve_rows(lay.Q, lay.K, spec.scale, spec.block, kept_g, lay.W, V, rows, lay.bias)
+    want = oracle.retrieve_rows(lay.Q, lay.K, spec.scale, spec.block, kept_g, lay.W, V, rows, lay.bias,
+                                renorm=renorm)
     got = O[:, :, rows].float().cpu().numpy() if reqs is None else O[reqs][:, :, rows].float().cpu().numpy()
     err = float(np.max(np.abs(got - want)))
     vmax = float(np.max(np.abs(V)))

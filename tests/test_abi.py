@@ -117,6 +117,11 @@ def test_retrieve_and_dense_reject_bad_arguments(mr):
     assert r(opts=mr.RetrieveOpts(-1, 4, 1)) == mr.MR_ERR_INVALID_ARG
     assert r(opts=mr.RetrieveOpts(0, 0, 2)) == mr.MR_ERR_INVALID_ARG      # 5 heads, groups of 2
     assert r(opts=mr.RetrieveOpts(0, 0, -1)) == mr.MR_ERR_INVALID_ARG
+    # paged values: pages of a positive multiple of 64 rows that cover the map's L = 512 rows
+    assert r(opts=mr.RetrieveOpts(0, 0, 1, fake, 32, 16)) == mr.MR_ERR_INVALID_ARG
+    assert r(opts=mr.RetrieveOpts(0, 0, 1, fake, 64, 7)) == mr.MR_ERR_INVALID_ARG      # 448 < 512 rows
+    assert r(opts=mr.RetrieveOpts(0, 0, 1, fake, 128, 0)) == mr.MR_ERR_INVALID_ARG
+    assert r(ve=64 * 64 * 5 - 1, opts=mr.RetrieveOpts(0, 0, 1, fake, 64, 8)) == mr.MR_ERR_INVALID_ARG  # no page fits
     # the workspace holds the status header and one progress counter per CTA (up to 1024)
     need = lib.mr_retrieve_workspace_bytes(ctypes.byref(b), 5, 64, 1)
     assert need == 256 + 1024 * 4

@@ -536,3 +536,62 @@ def test_fp8_full_size_headline_workload(mr):
     check_retrieve_status(mr, ws_r)
     rel = compare_retrieve(spec, lay, m, O, np.array([0, 5, spec.L // 2 + 17, spec.L - 1]), out_kind="fp8")
     print(spec.name, "fp8", stats, rel)
+
+
+@pytest.mark.parametrize("n,kw,page_rows", [(4, dict(L=1024, H_s=3, H_r=4), 64),        # key blocks span 2 pages
+                                            (2, dict(L=768, H_s=4, H_r=6), 128),
+                                            (2, dict(L=512, H_s=3, H_r=2, d_v=64), 64)])  # CUDA-core path
+def test_paged_values(mr, n, kw, page_rows):
+    """Values read through a per-request page table from a shuffled pool of pages
+    [page][H_v][page_rows][d_v] give the same outputs as the unpaged values."""
+    from cross_model_attention_mr_b200.workloads import Layer, round_to_bf16
+    spec = shrink(config(n), **kw)
+    lay = draw_layers(spec)[0]
+    n_req, L, H, dv = 2, spec.L, spec.H_r, spec.d_v
+    rng = np.random.default_rng(5)
+    V_req = round_to_bf16(rng.standard_normal((n_req, H, L, dv), dtype=np.float32))
+    ppr = L // page_rows
+    n_pages = n_req * ppr + 3                                   # a few pages no request uses
+    order = rng.permutation(n_pages)
+    table = order[: n_req * ppr].reshape(n_req, ppr).astype(np.int32)
+    pool = np.zeros((n_pages, H, page_rows, dv), np.float32)
+    for q in range(n_req):
+        for k in range(ppr):
+            pool[table[q, k]] = V_req[q][:, k * page_rows:(k + 1) * page_rows]
+    m = mr.compress(dev(lay.Q, "bf16"), dev(lay.K, "bf16"), p32(spec.p), spec.block,
+                    bias=mr.Bias.from_spec(lay.bias), scale=spec.scale)
+    ws_r = mr.Workspace(mr.retrieve_workspace_bytes(m, H, dv, n_req))
+    O = mr.retrieve(m, torch.from_numpy(lay.W).cuda(), dev(pool, "bf16"), n_req=n_req, ws=ws_r,
+                    v_pages=torch.from_numpy(table).cuda(), page_rows=page_rows)
+    torch.cuda.synchronize()
+    check_retrieve_status(mr, ws_r)
+    rows = np.array([0, 1, 63, 64, 200, L - 1])
+    for q in range(n_req):
+        lq = Layer(Q=lay.Q, K=lay.K, V=np.ascontiguousarray(V_req[q]), W=lay.W, bias=lay.bias)
+        compare_retrieve(spec, lq, m, O[q:q + 1], rows)
+
+
+@pytest.mark.parametrize("n,kw,map_dtype", [(2, dict(L=1024, H_s=4, H_r=5), None),            # tensor cores, block 64
+                                            (4, dict(L=1024, H_s=3, H_r=4), None),            # block 128
+                                            (4, dict(L=1024, H_s=3, H_r=4), "fp8"),
+                                            (1, {}, None)])                                   # fp32, CUDA cores
+def test_renormalised_maps(mr, n, kw, map_dtype):
+    """Each stored row divided by its kept mass: stored tiles and outputs against the oracle's
+    renormalised variant on the GPU's kept sets; the selection is the plain map's."""
+    spec = shrink(config(n), **kw) if kw else config(n)
+    lay = draw_layers(spec)[0]
+    Q, K = dev(lay.Q, spec.dtype), dev(lay.K, spec.dtype)
+    bias = mr.Bias.from_spec(lay.bias)
+    md = mr.MR_FP8_E4M3 if map_dtype == "fp8" else None
+    m = mr.compress(Q, K, p32(spec.p), spec.block, bias=bias, scale=spec.scale, store_mass=True, store_lse=True,
+                    map_dtype=md, renormalised=True)
+    plain = mr.compress(Q, K, p32(spec.p), spec.block, bias=bias, scale=spec.scale)
+    assert m.ws.sync_status() == mr.MR_OK
+    assert np.array_equal(m.kept_bits_host(), plain.kept_bits_host())
+    nqb = spec.L // spec.block
+    compare_compress(spec, lay, m, list(range(spec.H_s * nqb)), all_tiles=True, val_kind=map_dtype, renorm=True)
+    ws_r = mr.Workspace(mr.retrieve_workspace_bytes(m, spec.H_r, spec.d_v, 1))
+    O = mr.retrieve(m, torch.from_numpy(lay.W).cuda(), dev(lay.V, spec.dtype), ws=ws_r)
+    torch.cuda.synchronize()
+    check_retrieve_status(mr, ws_r)
+    compare_retrieve(spec, lay, m, O, np.arange(0, spec.L, 5), out_kind=map_dtype, renorm=True)
