@@ -4,11 +4,17 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/mr.h"
 #include "common.cuh"
 #include "kernels.h"
 
 using namespace mr;
+
+namespace mr {
+void debug_waits(uint64_t* wait_ns, int* skip_arrive);
+}
 
 namespace {
 
@@ -48,10 +54,18 @@ mr_status bias_ok(const mr_logit_bias* b, int keys) {
 
 mr_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MR_OK : MR_ERR_CUDA; }
 
+std::atomic<uint64_t> g_debug_wait_ns{0};
+std::atomic<int> g_debug_skip{0};
+
 // Clear the workspace header (status word and work-queue counters) in stream order.
 cudaError_t reset_header(void* ws, cudaStream_t st) { return cudaMemsetAsync(ws, 0, sizeof(WsHeader), st); }
 
 }  // namespace
+
+void mr::debug_waits(uint64_t* wait_ns, int* skip_arrive) {
+  *wait_ns = g_debug_wait_ns.load();
+  *skip_arrive = g_debug_skip.load();
+}
 
 extern "C" {
 
@@ -308,13 +322,22 @@ mr_status mr_bsr_export(const mr_bsr* map, int64_t n_tiles, float* out, void* st
   return from_cuda(launch_export(*map, n_tiles, out, (cudaStream_t)stream));
 }
 
-mr_status mr_gather_probe(const mr_bsr* map, int readers, void* ws, size_t ws_bytes, void* stream) {
+mr_status mr_gather_probe(const mr_bsr* map, int readers, int ring_slots, void* ws, size_t ws_bytes,
+                          void* stream) {
   if (!map || !ws || readers < 1 || readers > 1024 || ws_bytes < kWsHeaderBytes) return MR_ERR_INVALID_ARG;
+  if (ring_slots < 2 || ring_slots > 24 || ring_slots % 2) return MR_ERR_INVALID_ARG;
   if (!shape_ok(map->H_s, map->L, 64, map->block)) return MR_ERR_UNSUPPORTED;
   if (!map->row_ptr || !map->kept_bits || !map->vals) return MR_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
   if (reset_header(ws, st) != cudaSuccess) return MR_ERR_CUDA;
-  return from_cuda(launch_gather_probe(*map, readers, (WsHeader*)ws, st));
+  return from_cuda(launch_gather_probe(*map, readers, ring_slots, (WsHeader*)ws, st));
+}
+
+mr_status mr_debug_set(uint64_t wait_ns, int skip_arrive) {
+  if (skip_arrive < 0 || skip_arrive > 1) return MR_ERR_INVALID_ARG;
+  g_debug_wait_ns.store(wait_ns);
+  g_debug_skip.store(skip_arrive);
+  return MR_OK;
 }
 
 }  // extern "C"

@@ -109,9 +109,12 @@ __host__ __device__ __forceinline__ void tile_coords(int p, int B, int& a, int& 
   b = panel * P + ((pc ^ (a & 7)) * E) + (rem % E);
 }
 
-// Storage order of an fp8 (e4m3) tile: panels of 64 columns, rows of 64 bytes, no swizzle.
+// Storage order of an fp8 (e4m3) tile: panels of 64 columns, rows of 64 bytes, no swizzle; within
+// each group of 4 columns the bytes are ordered (0, 2, 1, 3), so one 32-bit word splits into the
+// half-precision pairs (0, 1) and (2, 3) with one mask and one shift each.
+__host__ __device__ __forceinline__ int fp8_perm4(int c) { return ((c & 1) << 1) | (c >> 1); }
 __host__ __device__ __forceinline__ int tile_offset_fp8(int a, int b, int B) {
-  return (b >> 6) * B * 64 + a * 64 + (b & 63);
+  return (b >> 6) * B * 64 + a * 64 + ((b & 63) & ~3) + fp8_perm4(b & 3);
 }
 // Scales per fp8 tile (one per 32-row x 64-column piece) and the index of element (a, b)'s scale.
 __host__ __device__ __forceinline__ int fp8_scales_per_tile(int B) { return (B / 32) * (B / 64); }

@@ -85,9 +85,16 @@ __device__ __forceinline__ void fail(Smem& s, const Params& p, uint32_t detail) 
   s.abort = 1;
 }
 
+// Unit k of the launch: heads in groups of kHeadGroup, each group's row blocks longest first,
+// the group's heads side by side.  The CTAs running at one time then share the K rows of a few
+// heads, which stay in L2, instead of streaming every head's K from DRAM for each row block.
+constexpr int kHeadGroup = 4;
 __device__ __forceinline__ void unit_of(const Params& p, int k, int& h, int& rb) {
-  rb = p.rb_hi - 1 - k / p.H;
-  h = k % p.H;
+  const int per_group = kHeadGroup * p.n_rb;
+  const int g = k / per_group, rem = k - g * per_group;
+  const int hg = min(kHeadGroup, p.H - g * kHeadGroup);  // heads in this group (the last may be short)
+  rb = p.rb_hi - 1 - rem / hg;
+  h = g * kHeadGroup + rem % hg;
 }
 
 // ------------------------------------------------------------------------------------------------

@@ -45,6 +45,8 @@ struct Params {
   Bias bias;
   __nv_bfloat16* O;
   WsHeader* ws;
+  uint64_t wait_ns;  // limit of the protocol waits (drains keep kTimeoutNs)
+  int skip_arrive;   // failure-path test: the softmax withholds its first "P ready" arrive
 };
 
 struct Smem {
@@ -111,7 +113,7 @@ __device__ void producer(Smem& s, const Params& p, const Tile& tl, int h, const 
   int j = 0;
   for (; j < tl.nk; ++j) {
     const int st = j & 1;
-    if (j >= 2 && !mbar_wait_sleep(&s.kv_empty[st], ((j >> 1) - 1) & 1, &s.abort, kTimeoutNs, 64)) {
+    if (j >= 2 && !mbar_wait_sleep(&s.kv_empty[st], ((j >> 1) - 1) & 1, &s.abort, p.wait_ns, 64)) {
       fail(s, p, 0x901);
       break;
     }
@@ -139,15 +141,15 @@ __device__ void mma_issuer(Smem& s, const Params& p, const Tile& tl) {
   const uint32_t id_pv = idesc_bf16_f32(128, 128, false, true);
   const uint32_t tbase = s.tmem_base;
   const uint32_t o_col = 256;
-  bool ok = mbar_wait(&s.q_full, 0, &s.abort, kTimeoutNs);
+  bool ok = mbar_wait(&s.q_full, 0, &s.abort, p.wait_ns);
   if (!ok) fail(s, p, 0x911);
   const uint32_t qa[2] = {smem_u32(&s.q[0][0]), smem_u32(&s.q[1][0])};
 
   // O += P_i V_i once the softmax has written P_i
   auto pv = [&](int i) -> bool {
     const int b = i & 1;
-    if (!mbar_wait(&s.p_full[b], (i >> 1) & 1, &s.abort, kTimeoutNs) ||
-        !mbar_wait(&s.v_full[b], (i >> 1) & 1, &s.abort, kTimeoutNs))
+    if (!mbar_wait(&s.p_full[b], (i >> 1) & 1, &s.abort, p.wait_ns) ||
+        !mbar_wait(&s.v_full[b], (i >> 1) & 1, &s.abort, p.wait_ns))
       return false;
     tc_fence_after();
     const uint32_t pa[2] = {smem_u32(&s.p[b][0][0]), smem_u32(&s.p[b][1][0])};
@@ -165,8 +167,8 @@ __device__ void mma_issuer(Smem& s, const Params& p, const Tile& tl) {
 
   for (int j = 0; j < tl.nk && ok; ++j) {
     const int b = j & 1;
-    if (!mbar_wait(&s.k_full[b], (j >> 1) & 1, &s.abort, kTimeoutNs) ||
-        (j >= 2 && !mbar_wait(&s.s_empty[b], ((j >> 1) - 1) & 1, &s.abort, kTimeoutNs))) {
+    if (!mbar_wait(&s.k_full[b], (j >> 1) & 1, &s.abort, p.wait_ns) ||
+        (j >= 2 && !mbar_wait(&s.s_empty[b], ((j >> 1) - 1) & 1, &s.abort, p.wait_ns))) {
       fail(s, p, 0x912);
       ok = false;
       break;
@@ -219,7 +221,7 @@ __device__ void softmax_group(Smem& s, const Params& p, const Tile& tl, int h) {
   bool ok = true;
   for (int j = 0; j < tl.nk; ++j) {
     const int b = j & 1;
-    if (!mbar_wait(&s.s_full[b], (j >> 1) & 1, &s.abort, kTimeoutNs)) {
+    if (!mbar_wait(&s.s_full[b], (j >> 1) & 1, &s.abort, p.wait_ns)) {
       fail(s, p, 0x921);
       ok = false;
       break;
@@ -277,7 +279,7 @@ __device__ void softmax_group(Smem& s, const Params& p, const Tile& tl, int h) {
         // P_{j-1} V_{j-1} has completed when its P buffer is released.  That buffer's earlier
         // completion (tile j - 3) was waited for before P_{j-1} was written and tile j + 1's
         // cannot happen before this warpgroup writes P_{j+1}, so the parity names one phase.
-        if (!mbar_wait(&s.p_empty[(j - 1) & 1], ((j - 1) >> 1) & 1, &s.abort, kTimeoutNs)) {
+        if (!mbar_wait(&s.p_empty[(j - 1) & 1], ((j - 1) >> 1) & 1, &s.abort, p.wait_ns)) {
           fail(s, p, 0x922);
           ok = false;
           break;
@@ -299,7 +301,7 @@ __device__ void softmax_group(Smem& s, const Params& p, const Tile& tl, int h) {
       ref = nref;
     }
     // P_j = 2^(s' - ref) as bf16 into the operand buffer this tile uses
-    if (j >= 2 && !mbar_wait(&s.p_empty[b], ((j >> 1) - 1) & 1, &s.abort, kTimeoutNs)) {
+    if (j >= 2 && !mbar_wait(&s.p_empty[b], ((j >> 1) - 1) & 1, &s.abort, p.wait_ns)) {
       fail(s, p, 0x923);
       ok = false;
       break;
@@ -327,11 +329,11 @@ __device__ void softmax_group(Smem& s, const Params& p, const Tile& tl, int h) {
     l += sum;
     fence_proxy_async_smem();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&s.p_full[b]);
+    if (lane == 0 && !(p.skip_arrive && j == 0)) mbar_arrive(&s.p_full[b]);
   }
   if (!ok) return;
   // epilogue: O / l -> bf16 -> global
-  if (!mbar_wait(&s.o_full, 0, &s.abort, kTimeoutNs)) {
+  if (!mbar_wait(&s.o_full, 0, &s.abort, p.wait_ns)) {
     fail(s, p, 0x924);
     return;
   }
@@ -426,6 +428,8 @@ cudaError_t tc_dense(const DenseArgs& a) {
   p.bias = a.bias;
   p.O = (__nv_bfloat16*)a.O;
   p.ws = a.ws;
+  debug_waits(&p.wait_ns, &p.skip_arrive);
+  if (p.wait_ns == 0) p.wait_ns = kTimeoutNs;
   CUtensorMap tq, tk, tv;
   if (!make_tmap_bf16_2d(&tq, a.Q, 128, (uint64_t)a.H * a.total_q, 256, 64, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tk, a.K, 128, (uint64_t)a.H * a.total_k, 256, 64, 128)) return cudaErrorInvalidValue;

@@ -66,9 +66,16 @@ __device__ __forceinline__ void fail(Smem& s, const Params& p, uint32_t detail) 
   s.abort = 1;
 }
 
+// Unit k of the launch: heads in groups of kHeadGroup, each group's row blocks longest first,
+// the group's heads side by side.  The CTAs running at one time then share the K rows of a few
+// heads, which stay in L2, instead of streaming every head's K from DRAM for each row block.
+constexpr int kHeadGroup = 4;
 __device__ __forceinline__ void unit_of(const Params& p, int k, int& h, int& rb) {
-  rb = p.rb_hi - 1 - k / p.H;
-  h = k % p.H;
+  const int per_group = kHeadGroup * p.n_rb;
+  const int g = k / per_group, rem = k - g * per_group;
+  const int hg = min(kHeadGroup, p.H - g * kHeadGroup);  // heads in this group (the last may be short)
+  rb = p.rb_hi - 1 - rem / hg;
+  h = g * kHeadGroup + rem % hg;
 }
 
 // One query block's kept bits, walked with non-decreasing J: kept flag, and the BSR position of
@@ -342,7 +349,7 @@ __device__ void emit_group(Smem& s, const Params& p, int w) {
               const int x = 16 * c16 + 4 * e;
               const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(pr[x] * inv, pr[x + 1] * inv), __NV_SATFINITE, __NV_E4M3);
               const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(pr[x + 2] * inv, pr[x + 3] * inv), __NV_SATFINITE, __NV_E4M3);
-              pk[e] = lo | (hi << 16);
+              pk[e] = __byte_perm(lo, hi, 0x5140);  // bytes of keys (0, 2, 1, 3)
             }
             *reinterpret_cast<uint4*>(dst + 16 * c16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }

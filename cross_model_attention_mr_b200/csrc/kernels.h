@@ -74,12 +74,16 @@ cudaError_t tc_retrieve(const RetrieveArgs& a);
 bool tc_dense_supported(const DenseArgs& a);
 cudaError_t tc_dense(const DenseArgs& a);
 
+// Failure-path test hook (mr_debug_set): wait limit for the dense kernel's protocol waits (0 = the
+// default 2 s) and whether its softmax withholds its first "P ready" arrive.
+void debug_waits(uint64_t* wait_ns, int* skip_arrive);
+
 // Shared by every compress path: exclusive scan of the kept counts into row_ptr, nnz, capacity.
 cudaError_t launch_scan_counts(const int* count, int n, mr_bsr map, WsHeader* ws, cudaStream_t st);
 
 cudaError_t launch_export(const mr_bsr& map, int64_t n_tiles, float* out, cudaStream_t st);
 
 // Measurement: the retrieval's map reads alone (each kept tile moved to shared memory `readers` times).
-cudaError_t launch_gather_probe(const mr_bsr& map, int readers, WsHeader* ws, cudaStream_t st);
+cudaError_t launch_gather_probe(const mr_bsr& map, int readers, int ring_slots, WsHeader* ws, cudaStream_t st);
 
 }  // namespace mr

@@ -16,7 +16,7 @@ namespace mr {
 namespace {
 
 constexpr int kThreads = 512;
-constexpr int kRing = 8;  // 16-byte slots per thread
+constexpr int kMaxRing = 24;  // 16-byte slots per thread at most (192 KB of shared memory)
 
 __device__ __forceinline__ void cp16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -25,8 +25,8 @@ __device__ __forceinline__ void cp16(uint32_t dst, const void* src) {
 __global__ void __launch_bounds__(kThreads, 1)
     k_gather_probe(const uint32_t* __restrict__ kept_bits, const int32_t* __restrict__ row_ptr, const char* vals,
                    int64_t capacity, int H_s, int nqb, int nkw, int B, int64_t tile_bytes, int readers,
-                   unsigned long long* sink) {
-  extern __shared__ uint4 ring_raw[];  // [kRing][kThreads] 16-byte slots
+                   int ring_slots, unsigned long long* sink) {
+  extern __shared__ uint4 ring_raw[];  // [ring_slots][kThreads] 16-byte slots
   uint4 (*ring)[kThreads] = reinterpret_cast<uint4 (*)[kThreads]>(ring_raw);
   __shared__ uint32_t list[64];
   __shared__ int n_list;
@@ -68,8 +68,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const char* tile = vals + (int64_t)list[k] * tile_bytes;
           for (int pc = tid; pc < pieces; pc += kThreads) {
             cp16(my + slot * (uint32_t)(kThreads * 16), tile + (int64_t)pc * 16);
-            slot = (slot + 1) % kRing;
-            if (++issued % 4 == 0) {
+            slot = slot + 1 == (uint32_t)ring_slots ? 0u : slot + 1;
+            // groups of half the ring: at most the whole ring in flight, never a slot reused early
+            if (++issued % (uint32_t)(ring_slots / 2) == 0) {
               asm volatile("cp.async.commit_group;" ::: "memory");
               asm volatile("cp.async.wait_group 1;" ::: "memory");
             }
@@ -87,7 +88,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_gather_probe(const mr_bsr& map, int readers, WsHeader* ws, cudaStream_t st) {
+cudaError_t launch_gather_probe(const mr_bsr& map, int readers, int ring_slots, WsHeader* ws, cudaStream_t st) {
+  if (ring_slots < 2 || ring_slots > kMaxRing || ring_slots % 2) return cudaErrorInvalidValue;
   const int nqb = map.L / map.block;
   const int64_t tile_bytes = (int64_t)map.block * map.block * (map.val_dtype == MR_BF16 ? 2 : map.val_dtype == MR_F32 ? 4 : 1);
   int dev = 0, sms = 148;
@@ -95,13 +97,13 @@ cudaError_t launch_gather_probe(const mr_bsr& map, int readers, WsHeader* ws, cu
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int n_units = ((map.L + 127) / 128) * readers;
   const int grid = n_units < sms ? n_units : sms;
-  const size_t smem = (size_t)kRing * kThreads * 16;
+  const size_t smem = (size_t)ring_slots * kThreads * 16;
   cudaError_t e = cudaFuncSetAttribute(k_gather_probe, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps(kKGatherProbe, st);
   k_gather_probe<<<grid, kThreads, smem, st>>>(map.kept_bits, map.row_ptr, (const char*)map.vals, map.capacity_tiles,
                                             map.H_s, nqb, (nqb + 31) / 32, map.block, tile_bytes, readers,
-                                            reinterpret_cast<unsigned long long*>(&ws->counters[0]));
+                                            ring_slots, reinterpret_cast<unsigned long long*>(&ws->counters[0]));
   return cudaGetLastError();
 }
 

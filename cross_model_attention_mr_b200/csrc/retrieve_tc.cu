@@ -101,6 +101,7 @@ constexpr uint32_t kUnitEnd = 1u, kEmptyUnit = 2u, kEnd = 4u;
 // in its normal range; a mixed value is at most 2^14), undone exactly in the epilogue.
 constexpr int kPieces8 = 1;
 constexpr float kF8Pre = 16384.f;
+constexpr float kF8Decode = 256.f;  // the integer decode yields value * 2^-8
 
 template <bool F8>
 struct SmemT {
@@ -552,10 +553,17 @@ __device__ __forceinline__ float lds32f(uint32_t addr) {
   asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
   return v;
 }
-// two e4m3 values (low byte = lower column) -> half2
-__device__ __forceinline__ __half2 e4m3x2_to_half2(uint32_t two) {
-  const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
-  return *reinterpret_cast<const __half2*>(&r);
+// A stored word holds the e4m3 codes of keys (0, 2, 1, 3) of a group of four, all non-negative.
+// Placing a code's 7 bits at bits 7..13 of a half gives exactly its value times 2^-8 (the exponent
+// biases are 7 and 15; subnormals line up too), so a word splits into the half pairs of keys (0, 1)
+// and (2, 3) with a mask and a shift each.
+__device__ __forceinline__ __half2 e4m3_pair01(uint32_t w) {
+  const uint32_t h = (w & 0x007F007Fu) << 7;
+  return *reinterpret_cast<const __half2*>(&h);
+}
+__device__ __forceinline__ __half2 e4m3_pair23(uint32_t w) {
+  const uint32_t h = (w >> 1) & 0x3F803F80u;
+  return *reinterpret_cast<const __half2*>(&h);
 }
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
@@ -682,7 +690,7 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
 
   // fp8 entry: acch[g] += (W[r_g, s] * scale * 2^14) * (the thread's 16 e4m3 values)
   auto mix_entry8 = [&](const Entry& E, uint32_t data, uint32_t sdata) {
-    const float sc = lds32f(sdata) * kF8Pre;
+    const float sc = lds32f(sdata) * (kF8Pre * kF8Decode);
     __half2 w2[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) w2[g] = __float2half2_rn(E.w[g] * sc);
@@ -690,7 +698,7 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
     const uint32_t wd[4] = {d.x, d.y, d.z, d.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const __half2 lo = e4m3x2_to_half2(wd[e]), hi = e4m3x2_to_half2(wd[e] >> 16);
+      const __half2 lo = e4m3_pair01(wd[e]), hi = e4m3_pair23(wd[e]);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         acch[g][2 * e] = __hfma2(w2[g], lo, acch[g][2 * e]);

@@ -292,7 +292,7 @@ struct MapVals<uint8_t> {
   __device__ __forceinline__ void coords(int off, int B, int& a, int& b) const {
     const int panel = off / (B * 64), rem = off - panel * B * 64;
     a = rem >> 6;
-    b = panel * 64 + (rem & 63);
+    b = panel * 64 + ((rem & 63) & ~3) + fp8_perm4(rem & 3);  // the order (0, 2, 1, 3) is its own inverse
   }
   __device__ __forceinline__ float at(int64_t t, int off, int B) const {
     int a, b;

@@ -75,7 +75,8 @@ EXPORTS = {
     "mr_bm_release": ([_c_p, _c_i64], ctypes.c_int),
     "mr_bm_evicted": ([_c_p, ctypes.POINTER(_c_i64), ctypes.c_int], ctypes.c_int),
     "mr_bm_stats": ([_c_p, ctypes.POINTER(_c_i64)], ctypes.c_int),
-    "mr_gather_probe": ([ctypes.POINTER(BSR), ctypes.c_int, _c_p, _c_sz, _c_p], ctypes.c_int),
+    "mr_gather_probe": ([ctypes.POINTER(BSR), ctypes.c_int, ctypes.c_int, _c_p, _c_sz, _c_p], ctypes.c_int),
+    "mr_debug_set": ([ctypes.c_uint64, ctypes.c_int], ctypes.c_int),
     "mr_profile_enable": ([ctypes.c_int], ctypes.c_int),
     "mr_profile_read": ([_c_p, _c_p, ctypes.c_int], ctypes.c_int),
     "mr_kernel_name": ([ctypes.c_int], ctypes.c_char_p),
@@ -421,11 +422,12 @@ def dense_ref(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, cu_q: torch.Ten
     return out
 
 
-def gather_probe(m: "Map", readers: int, ws: Optional[Workspace] = None, stream=None) -> None:
+def gather_probe(m: "Map", readers: int, ws: Optional[Workspace] = None, stream=None, ring_slots: int = 8) -> None:
     """mr_gather_probe: the retrieval's map reads alone (measurement)."""
     if ws is None:
         ws = Workspace(256, m.vals.device)
-    check(LIB.mr_gather_probe(ctypes.byref(m.c), int(readers), ws.ptr, ws.nbytes, _stream(stream)), "mr_gather_probe")
+    check(LIB.mr_gather_probe(ctypes.byref(m.c), int(readers), int(ring_slots), ws.ptr, ws.nbytes, _stream(stream)),
+          "mr_gather_probe")
 
 
 def profile_enable(on: bool = True) -> bool:

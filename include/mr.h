@@ -92,8 +92,9 @@ typedef struct {
  *               (b / P) * block * P + a * P + E * (((b % P) / E) ^ (a % 8)) + b % E,
  *             E = 16 / sizeof(element).  (Each panel is a 128-byte-swizzled MMA operand.)
  *             MR_FP8_E4M3 tiles are stored in panels of 64 columns, each panel holding its `block`
- *             rows of 64 bytes in turn with no swizzle: element (a, b) at
- *               (b / 64) * block * 64 + a * 64 + b % 64,
+ *             rows of 64 bytes in turn with no swizzle, and within every group of 4 columns the
+ *             bytes ordered (0, 2, 1, 3): element (a, b) at
+ *               (b / 64) * block * 64 + a * 64 + (b % 64) - (b % 4) + perm(b % 4), perm = {0, 2, 1, 3},
  *             and the value is e4m3(a, b) * tile_scale[t * S + (a / 32) * (block / 64) + b / 64],
  *             S = (block / 32) * (block / 64) scales per tile.
  *             mr_bsr_export converts tiles to plain row-major fp32.
@@ -408,10 +409,22 @@ int64_t mr_kernel_launches(void);   /* kernels launched by this library in this 
  * the retrieval's order (128-row blocks longest first; key blocks J <= I; the kept tile of every
  * sender head) and moves each stored tile into shared memory `readers` times (by `readers` CTAs
  * working on the same row block side by side, as the retrieval's receiver-head groups do) with
- * 16-byte asynchronous copies, doing no arithmetic.  Time it on `stream`; bytes moved =
+ * 16-byte asynchronous copies, doing no arithmetic; each of its 512 threads keeps up to
+ * ring_slots copies in flight (even, 2 .. 24).  Time it on `stream`; bytes moved =
  * readers * stored tiles * tile bytes.  ws: at least 256 bytes (status header).
  */
-mr_status mr_gather_probe(const mr_bsr* map, int readers, void* ws, size_t ws_bytes, void* stream);
+mr_status mr_gather_probe(const mr_bsr* map, int readers, int ring_slots, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/*
+ * Failure-path test hook (not part of the method; process-wide, for tests).  Sets the limit of the
+ * tensor-core dense kernel's protocol waits to wait_ns (0 = the default 2 s) and, with
+ * skip_arrive = 1, makes its softmax warpgroup withhold its first "P ready" arrive, so the MMA
+ * warp's wait runs out: the call records MR_ERR_TIMEOUT (detail 0x913) in the workspace's status
+ * word, drains its copies and MMAs, frees Tensor Memory and returns, leaving the context usable.
+ * mr_debug_set(0, 0) restores normal operation.  No GPU fault is involved.
+ */
+mr_status mr_debug_set(uint64_t wait_ns, int skip_arrive);
 
 #ifdef __cplusplus
 }

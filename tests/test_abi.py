@@ -132,3 +132,10 @@ def test_retrieve_and_dense_reject_bad_arguments(mr):
     assert d(cu=None) == mr.MR_ERR_INVALID_ARG
     assert d(d=32) == mr.MR_ERR_UNSUPPORTED
     assert d(dt=3) == mr.MR_ERR_INVALID_ARG
+
+
+def test_debug_hook_validates_and_resets(mr):
+    lib = mr.LIB
+    assert lib.mr_debug_set(0, 2) == mr.MR_ERR_INVALID_ARG
+    assert lib.mr_debug_set(1000, 1) == mr.MR_OK
+    assert lib.mr_debug_set(0, 0) == mr.MR_OK

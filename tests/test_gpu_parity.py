@@ -470,7 +470,10 @@ def test_dense_tensor_core_ragged_with_key_block_bias(mr):
     for s, (lq, lk) in enumerate(seqs):
         if lq == 0:
             continue
-        want = oracle.dense_rows(Qs[s], Ks[s], Vs[s], 1.0 / np.sqrt(d), np.arange(lq), int(offs[s]), sb)
+        # the oracle's key-block table has exactly ceil(keys / kb_block) columns per head
+        sbs = SpecBias(sink_len=16, sink_bias=3.0, window=128, window_bias=3.0,
+                       kb_bias=np.ascontiguousarray(kb[:, : (lk + 63) // 64]), kb_block=64)
+        want = oracle.dense_rows(Qs[s], Ks[s], Vs[s], 1.0 / np.sqrt(d), np.arange(lq), int(offs[s]), sbs)
         err = np.max(np.abs(Oh[:, cu_q[s]:cu_q[s + 1]] - want))
         assert err <= OUT_TOL["bf16"] * float(np.abs(Vs[s]).max()), (s, err)
 
