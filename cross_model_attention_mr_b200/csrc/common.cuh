@@ -26,6 +26,22 @@ __device__ __forceinline__ void set_status(WsHeader* ws, uint32_t code, uint32_t
   if (atomicCAS(&ws->status, 0u, code) == 0u) ws->detail = detail;
 }
 
+// Bounds-checked build (libmr_checked.so, compiled with -DMR_CHECKED): the tensor-core kernels
+// check the index of every global store, and of every map read whose index comes from device
+// data, against the extent the host passed.  A miss records MR_ERR_DEVICE_CHECK with the site's
+// code (0xC..) and skips the access.  In the normal build the check is compiled out; the checks
+// that are always on (capacity, value offsets and pages) stay in both.
+#ifdef MR_CHECKED
+constexpr bool kCheckedBuild = true;
+__device__ __forceinline__ bool checked(WsHeader* ws, bool ok, uint32_t site) {
+  if (!ok) set_status(ws, MR_ERR_DEVICE_CHECK, site);
+  return ok;
+}
+#else
+constexpr bool kCheckedBuild = false;
+__device__ __forceinline__ bool checked(WsHeader*, bool, uint32_t) { return true; }
+#endif
+
 // Logit bias b(h, i, j) for a causal pair j <= i: the largest applicable term, 0 if none.
 // (Synthetic stand-in for sink / local-window / retrieval-head structure.)
 struct Bias {

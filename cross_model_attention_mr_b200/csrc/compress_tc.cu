@@ -193,13 +193,19 @@ __device__ __forceinline__ float warp_max32(const float (&v)[32]) {
   return m[0];
 }
 
-// Sum of 2^x over 32 values with 8 independent partial sums.
+// Sum of 2^x over 32 values with 8 independent partial sums.  The values kEmuMask names (bit k:
+// value 8 m + k) take the FMA-pipe exponential of degree 5, the rest the multi-function unit,
+// whose 16 results per clock per SM otherwise bound this kernel.
+constexpr uint32_t kEmuMask = 0x88;
+__device__ __forceinline__ float ex2_mixed(float x, int t) {
+  return ((kEmuMask >> (t & 7)) & 1) ? ex2_poly<5>(x) : ex2_approx(x);
+}
 __device__ __forceinline__ float sum_ex2_32(const float (&x)[32]) {
   float a[8];
 #pragma unroll
-  for (int t = 0; t < 8; ++t) a[t] = ex2_approx(x[t]);
+  for (int t = 0; t < 8; ++t) a[t] = ex2_mixed(x[t], t);
 #pragma unroll
-  for (int t = 8; t < 32; ++t) a[t & 7] += ex2_approx(x[t]);
+  for (int t = 8; t < 32; ++t) a[t & 7] += ex2_mixed(x[t], t);
   return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
 
@@ -353,7 +359,7 @@ __device__ void softmax_group(Smem& s, const Params& p, int w) {
       if (co != -INFINITY) Ls += lo * ex2_approx(co - C);
     }
     const float lse2 = C + __log2f(Ls);
-    if (w == 0 && row_ok && good) {
+    if (w == 0 && row_ok && good && checked(p.ws, h < p.H && i < p.L, 0xC11)) {
       const size_t gi = (size_t)h * p.L + i;
       p.lse_ws[gi] = lse2 * kLn2;
       if (p.lse_out) p.lse_out[gi] = lse2 * kLn2;
@@ -365,13 +371,23 @@ __device__ void softmax_group(Smem& s, const Params& p, int w) {
       uint32_t xs[32];
       tmem_ld32(tbase + lane_addr + xbase + c0, xs);
       tmem_wait_ld();
+      float v[32];
 #pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        float x = __uint_as_float(xs[t]) * scale;
+      for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(xs[t]) * scale;
+      // sum each of the 32 columns over the warp's 32 rows: every step hands half of the columns
+      // still held to the partner lane and adds the other half, so after five steps lane l holds
+      // the sum of column l (31 shuffles instead of 5 per column)
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-        if (lane == t && c0 + t < used) s.red[w][q4][c0 + t] = x;
+      for (int o = 16, n = 32; o >= 1; o >>= 1, n >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int t = 0; t < n / 2; ++t) {
+          const float send = upper ? v[t] : v[t + n / 2];
+          const float keep = upper ? v[t + n / 2] : v[t];
+          v[t] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
       }
+      if (c0 + lane < used) s.red[w][q4][c0 + lane] = v[0];
     }
     named_sync(1, 256);
     // block masses: own columns -> key blocks
@@ -457,13 +473,15 @@ __device__ void softmax_group(Smem& s, const Params& p, int w) {
       for (int t = gtid; t < kstar; t += 128) atomicOr(&s.bits[w][s.sorted[w][t] >> 5], 1u << (s.sorted[w][t] & 31));
       named_sync(bar_id, 128);
       const int u = h * p.nqb + I;
-      if (gtid < p.nkw) p.kept_bits[(size_t)u * p.nkw + gtid] = s.bits[w][gtid];
-      if (gtid == 0) {
-        p.count_ws[u] = kstar;
-        p.kept_mass[u] = s.kmass[w];
+      if (checked(p.ws, h < p.H && I >= 0 && I < p.nqb, 0xC12)) {
+        if (gtid < p.nkw) p.kept_bits[(size_t)u * p.nkw + gtid] = s.bits[w][gtid];
+        if (gtid == 0) {
+          p.count_ws[u] = kstar;
+          p.kept_mass[u] = s.kmass[w];
+        }
+        if (p.mass_out)
+          for (int J = gtid; J < p.nqb; J += 128) p.mass_out[(size_t)u * p.nqb + J] = J <= I ? m[J] : 0.f;
       }
-      if (p.mass_out)
-        for (int J = gtid; J < p.nqb; J += 128) p.mass_out[(size_t)u * p.nqb + J] = J <= I ? m[J] : 0.f;
     }
     named_sync(1, 256);  // the shared arrays are reused by the next unit
     if (p.renorm) {

@@ -364,6 +364,7 @@ __device__ void emit_group(Smem& s, const Params& p, int w) {
           const int piece = p.B == 128 ? 0 : 2 * rh + hh;
           const int64_t t = tpos[piece];
           if (t >= p.capacity) continue;
+          if (!checked(p.ws, t >= 0 && (p.B == 128 ? T : 2 * T + hh) < p.nqb, 0xC21)) continue;
           // destination: panel hh of the 128-tile, or the (rh, hh) 64-tile; this warp's 32 rows
           if (!F8) {
             const int64_t tbytes = (int64_t)p.B * p.B * 2;

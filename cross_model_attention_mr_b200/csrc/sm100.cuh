@@ -141,6 +141,16 @@ __device__ __forceinline__ void tmem_relinquish() {
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
+// Per-warpgroup register limits (every warp of a warpgroup executes the same one).  The limits
+// of all warpgroups together must stay within the block's launch allocation, or an increase waits.
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -191,6 +201,35 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe, to take part of the exponentials off the multi-function unit.  Range
+// reduction x = n + f with n the integer nearest x (adding 1.5 * 2^23 leaves n in the low mantissa
+// bits) and f in [-1/2, 1/2]; 2^f from a polynomial whose coefficients were fitted by iteratively
+// reweighted least squares for the smallest relative error on that interval; n is added to the
+// exponent field.  Degree 3: relative error at most 7.5e-5 (for values rounded to bf16 next);
+// degree 5: at most 2.4e-7 in fp32, the multi-function unit's own accuracy class.  Inputs below
+// -125 give 0 (masked keys among them); callers keep inputs at most 8, far from overflow.
+template <int Deg>
+__device__ __forceinline__ float ex2_poly(float x) {
+  static_assert(Deg == 3 || Deg == 5, "degree 3 or 5");
+  const float xc = fmaxf(x, -127.f);
+  const float t = __fadd_rn(xc, 12582912.f);
+  const float f = __fsub_rn(xc, __fsub_rn(t, 12582912.f));
+  float p;
+  if (Deg == 3) {
+    p = fmaf(f, 0.0551716648f, 0.242611125f);
+    p = fmaf(p, f, 0.693260968f);
+    p = fmaf(p, f, 0.999928057f);
+  } else {
+    p = fmaf(f, 0.00132764713f, 0.00967554096f);
+    p = fmaf(p, f, 0.0555071309f);
+    p = fmaf(p, f, 0.240221202f);
+    p = fmaf(p, f, 0.693146944f);
+    p = fmaf(p, f, 1.00000012f);
+  }
+  const float y = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  return x < -125.f ? 0.f : y;
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
