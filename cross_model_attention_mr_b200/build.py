@@ -13,6 +13,9 @@ CSRC = os.path.join(PKG, "csrc")
 ROOT = os.path.dirname(PKG)
 OUT = os.path.join(PKG, "libmr.so")
 OBJ_DIR = os.path.join(PKG, "_build")
+# the bounds-checked build: same sources with -DMR_CHECKED
+OUT_CHECKED = os.path.join(PKG, "libmr_checked.so")
+OBJ_DIR_CHECKED = os.path.join(PKG, "_build_checked")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
@@ -42,15 +45,19 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build_library(force: bool = False, verbose: bool = False, extra: list | None = None) -> str:
-    os.makedirs(OBJ_DIR, exist_ok=True)
+def build_library(force: bool = False, verbose: bool = False, extra: list | None = None,
+                  checked: bool = False) -> str:
+    """Compile every source under csrc/ and link libmr.so (or, with ``checked``, the bounds-checked
+    libmr_checked.so from its own object folder).  Only stale objects are rebuilt."""
+    out, obj_dir = (OUT_CHECKED, OBJ_DIR_CHECKED) if checked else (OUT, OBJ_DIR)
+    os.makedirs(obj_dir, exist_ok=True)
     srcs, hdrs = _sources(), _headers()
     cc = nvcc()
-    flags = ARCH + FLAGS + (extra or [])
+    flags = ARCH + FLAGS + (["-DMR_CHECKED"] if checked else []) + (extra or [])
     objs = []
     jobs = []
     for s in srcs:
-        o = os.path.join(OBJ_DIR, os.path.basename(s) + ".o")
+        o = os.path.join(obj_dir, os.path.basename(s) + ".o")
         objs.append(o)
         if force or _stale(o, [s] + hdrs):
             jobs.append([cc, *flags, "-c", s, "-o", o])
@@ -65,12 +72,12 @@ def build_library(force: bool = False, verbose: bool = False, extra: list | None
 
     with cf.ThreadPoolExecutor(max_workers=min(8, max(1, len(jobs)))) as ex:
         list(ex.map(run, jobs))
-    if force or jobs or _stale(OUT, objs):
-        tmp = OUT + f".tmp{os.getpid()}"
+    if force or jobs or _stale(out, objs):
+        tmp = out + f".tmp{os.getpid()}"
         run([cc, *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static", "-ldl", "-lrt", "-lpthread"])
-        os.replace(tmp, OUT)
-    return OUT
+        os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
-    print(build_library(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build_library(force="--force" in sys.argv, verbose="-v" in sys.argv, checked="--checked" in sys.argv))

@@ -85,6 +85,8 @@ const char* mr_status_string(mr_status s) {
   return "unknown status";
 }
 
+int mr_checked_build(void) { return mr::kCheckedBuild ? 1 : 0; }
+
 int mr_device_supported(void) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;

@@ -792,7 +792,7 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
         uint32_t v[16];
         tmem_ld16(tbase + ((uint32_t)(32 * tw) << 16) + 128 * a + 16 * cc, v);
         tmem_wait_ld();
-        if (valid && row_out) {
+        if (valid && row_out && checked(p.ws, q < p.n_req && r < p.H_r && i < p.L, 0xC31)) {
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             uint32_t pk[4];

@@ -16,7 +16,10 @@ from typing import Optional
 import numpy as np
 import torch
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmr.so")
+# MR_LIBRARY=checked selects the bounds-checked build (libmr_checked.so): same API and results,
+# with every global store of the tensor-core kernels checked against its extent on the device.
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                        "libmr_checked.so" if os.environ.get("MR_LIBRARY") == "checked" else "libmr.so")
 
 MR_OK, MR_ERR_INVALID_ARG, MR_ERR_UNSUPPORTED, MR_ERR_CAPACITY = 0, 1, 2, 3
 MR_ERR_CUDA, MR_ERR_TIMEOUT, MR_ERR_DEVICE_CHECK, MR_ERR_RANGE = 4, 5, 6, 7
@@ -46,6 +49,7 @@ EXPORTS = {
     "mr_version": ([], ctypes.c_int),
     "mr_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "mr_device_supported": ([], ctypes.c_int),
+    "mr_checked_build": ([], ctypes.c_int),
     "mr_compress_workspace_bytes": ([ctypes.c_int] * 4, _c_sz),
     "mr_bsr_max_tiles": ([ctypes.c_int] * 3, _c_i64),
     "mr_compress": ([_c_p, _c_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _c_f32, _c_f32,
@@ -213,6 +217,22 @@ class Map:
         w = self.kept_bits.cpu().numpy().view(np.uint32).reshape(self.H_s, self.nqb, self.nkw)
         bits = ((w[..., :, None] >> np.arange(32, dtype=np.uint32)) & 1).astype(np.uint8)
         return bits.reshape(self.H_s, self.nqb, self.nkw * 32)[..., : self.nqb]
+
+    def to(self, device) -> "Map":
+        """A copy of this map on `device` (same capacity and flags), e.g. to move a received map
+        from host memory onto the GPU that retrieves from it."""
+        m = Map(self.H_s, self.L, self.block, self.dtype, max(1, self.capacity), device, self.mass is not None,
+                self.lse is not None, bool(self.c.renormalised))
+        m.capacity = self.capacity
+        m.c.capacity_tiles = self.capacity
+        pairs = [(m.row_ptr, self.row_ptr), (m.col_idx, self.col_idx), (m.vals, self.vals),
+                 (m.kept_mass, self.kept_mass), (m.kept_bits, self.kept_bits), (m.nnz, self.nnz)]
+        for opt in ("mass", "lse", "tile_scale"):
+            if getattr(self, opt) is not None:
+                pairs.append((getattr(m, opt), getattr(self, opt)))
+        for dst, src in pairs:
+            dst.copy_(src)
+        return m
 
     def export(self, n_tiles: Optional[int] = None, stream=None) -> torch.Tensor:
         n = self.nnz_host(stream) if n_tiles is None else int(n_tiles)

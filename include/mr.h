@@ -139,6 +139,14 @@ const char* mr_status_string(mr_status s);
 int mr_device_supported(void);
 
 /*
+ * 1 in the bounds-checked build of the library (libmr_checked.so), else 0.  That build checks the
+ * index of every global store of the tensor-core kernels, and of every map read whose index comes
+ * from device data, against the extents passed in; a miss skips the access and records
+ * MR_ERR_DEVICE_CHECK with a site code in the workspace status.  Same entry points and results.
+ */
+int mr_checked_build(void);
+
+/*
  * Workspace bytes mr_compress needs for this shape (device memory, 256-byte aligned, contents
  * need no initialisation).  Returns 0 for an unsupported shape.
  */

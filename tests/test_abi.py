@@ -37,6 +37,22 @@ def test_library_exports_every_declared_symbol(mr):
     assert set(declared_functions()) <= set(mr.EXPORTS)
 
 
+def test_checked_build_exports_the_same_symbols(mr):
+    """libmr_checked.so (compiled with -DMR_CHECKED) is a drop-in twin of libmr.so."""
+    path = os.path.join(os.path.dirname(mr.LIB_PATH), "libmr_checked.so")
+    assert os.path.exists(path), "build it with __graft_entry__.build()"
+    lib = ctypes.CDLL(path)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    lib.mr_checked_build.restype = ctypes.c_int
+    assert lib.mr_checked_build() == 1
+
+
+def test_library_variant_matches_environment(mr):
+    """MR_LIBRARY=checked loads the bounds-checked build; anything else the normal one."""
+    assert mr.LIB.mr_checked_build() == (1 if os.environ.get("MR_LIBRARY") == "checked" else 0)
+
+
 def test_status_strings(mr):
     for code in range(8):
         s = mr.LIB.mr_status_string(code)
