@@ -37,6 +37,13 @@ constexpr int kThreads = 384;
 constexpr int kProducerWarp = 0;
 constexpr int kMmaWarp = 1;
 constexpr int kSoftmaxWarp0 = 4;  // warpgroup w = warps 4 + 4w .. 7 + 4w
+// Warpgroup 0 (producer, MMA warp, two idle warps) drops to 56 registers so the two softmax
+// warpgroups can rise to 224: each SM sub-partition holds one warp of each warpgroup, and
+// 56 + 2 x 224 is exactly the launch's 3 x 168.
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsControl = 56;
+constexpr int kRegsSoftmax = 224;
+static_assert(kRegsControl + 2 * kRegsSoftmax == 3 * kLaunchRegs, "register split");
 constexpr int kKStages = 4;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -253,80 +260,80 @@ __device__ void softmax_group(Smem& s, const Params& p, int w) {
       const int j_tile = 128 * T;
       const bool special = (T == rb) || (j_tile < p.bias.sink_len) ||
                            (p.bias.window > 0 && j_tile + 127 > 128 * rb - p.bias.window);
-      float acc[2] = {0.f, 0.f};
+      // the whole S tile of this row into registers, then the buffer goes back to the MMA warp at
+      // once, so the next tile's QK^T overlaps this tile's exponentials
+      float v[4][32];
+      {
+        uint32_t raw[4][32];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        // 64 logits of this row: keys j_tile + 64 hh .. + 63 (one key block when the block is 64)
-        float v[2][32];
-        {
-          uint32_t raw[2][32];
-          tmem_ld32(tbase + lane_addr + 128 * w + 64 * hh, raw[0]);
-          tmem_ld32(tbase + lane_addr + 128 * w + 64 * hh + 32, raw[1]);
+        for (int cc = 0; cc < 4; ++cc) tmem_ld32(tbase + lane_addr + 128 * w + 32 * cc, raw[cc]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+          for (int t = 0; t < 32; ++t) v[cc][t] = __uint_as_float(raw[cc][t]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.s_empty[w]);
+      float mc;
+      if (!special) {
+        // only the key-block term can apply: a constant per 32 keys
+        mc = -INFINITY;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) mc = fmaxf(mc, fmaf(warp_max32(v[cc]), p.a, kbo[cc]));
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int j0 = j_tile + 32 * cc;
+          const float kb = kb_term(p.bias, h, j0);
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const int j = j0 + t;
+            v[cc][t] = (row_ok && j <= i) ? fmaf(v[cc][t], p.a, bias_with_kb(p.bias, i, j, kb) * kLog2e) : -INFINITY;
+          }
+        }
+        mc = fmaxf(fmaxf(warp_max32(v[0]), warp_max32(v[1])), fmaxf(warp_max32(v[2]), warp_max32(v[3])));
+      }
+      if (!row_ok) mc = -INFINITY;
+      const bool need = mc > c + kRescale;
+      if (__any_sync(0xffffffffu, need)) {
+        const float cn = need ? mc : c;
+        const float f = need ? ex2_approx(c - cn) : 1.f;  // c = -inf gives 0
+        for (int c0 = 0; c0 < used; c0 += 32) {
+          uint32_t xs[32];
+          tmem_ld32(tbase + lane_addr + xbase + c0, xs);
           tmem_wait_ld();
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc)
-#pragma unroll
-            for (int t = 0; t < 32; ++t) v[cc][t] = __uint_as_float(raw[cc][t]);
+          for (int t = 0; t < 32; ++t) xs[t] = __float_as_uint(__uint_as_float(xs[t]) * f);
+          tmem_st32(tbase + lane_addr + xbase + c0, xs);
         }
-        if (hh == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&s.s_empty[w]);
-        }
-        const int j0 = j_tile + 64 * hh;
-        float off[2] = {0.f, 0.f};
-        float mc;
-        if (!special) {
-          // only the key-block term can apply: a constant per 32 keys
-          off[0] = kbo[2 * hh];
-          off[1] = kbo[2 * hh + 1];
-          mc = fmaxf(fmaf(warp_max32(v[0]), p.a, off[0]), fmaf(warp_max32(v[1]), p.a, off[1]));
-        } else {
+        tmem_wait_st();
+        c = cn;
+      }
+      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      if (c != -INFINITY && row_ok) {
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            const float kb = kb_term(p.bias, h, j0 + 32 * cc);
+        for (int cc = 0; cc < 4; ++cc) {
+          if (!special) {
+            const float o = kbo[cc] - c;
 #pragma unroll
-            for (int t = 0; t < 32; ++t) {
-              const int j = j0 + 32 * cc + t;
-              v[cc][t] = (row_ok && j <= i) ? fmaf(v[cc][t], p.a, bias_with_kb(p.bias, i, j, kb) * kLog2e) : -INFINITY;
-            }
+            for (int t = 0; t < 32; ++t) v[cc][t] = fmaf(v[cc][t], p.a, o);
+          } else {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) v[cc][t] -= c;  // -inf stays -inf and gives 0
           }
-          mc = fmaxf(warp_max32(v[0]), warp_max32(v[1]));
+          sum[cc] = sum_ex2_32(v[cc]);
         }
-        if (!row_ok) mc = -INFINITY;
-        const bool need = mc > c + kRescale;
-        if (__any_sync(0xffffffffu, need)) {
-          const float cn = need ? mc : c;
-          const float f = need ? ex2_approx(c - cn) : 1.f;  // c = -inf gives 0
-          acc[0] *= f;
-          acc[1] *= f;
-          for (int c0 = 0; c0 < used; c0 += 32) {
-            uint32_t xs[32];
-            tmem_ld32(tbase + lane_addr + xbase + c0, xs);
-            tmem_wait_ld();
-#pragma unroll
-            for (int t = 0; t < 32; ++t) xs[t] = __float_as_uint(__uint_as_float(xs[t]) * f);
-            tmem_st32(tbase + lane_addr + xbase + c0, xs);
-          }
-          tmem_wait_st();
-          c = cn;
-        }
-        float sum = 0.f;
-        if (c != -INFINITY && row_ok) {
-#pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            if (!special) {
-              const float o = off[cc] - c;
-#pragma unroll
-              for (int t = 0; t < 32; ++t) v[cc][t] = fmaf(v[cc][t], p.a, o);
-            } else {
-#pragma unroll
-              for (int t = 0; t < 32; ++t) v[cc][t] -= c;  // -inf stays -inf and gives 0
-            }
-            sum += sum_ex2_32(v[cc]);
-          }
-        }
-        acc[(p.B == 64) ? hh : 0] += sum;
+      }
+      // block sums of this tile: one 128-key block, or two 64-key blocks
+      float acc[2];
+      if (p.B == 64) {
+        acc[0] = sum[0] + sum[1];
+        acc[1] = sum[2] + sum[3];
+      } else {
+        acc[0] = (sum[0] + sum[1]) + (sum[2] + sum[3]);
+        acc[1] = 0.f;
       }
       if (per_tile == 1)
         tmem_st1(tbase + lane_addr + xbase + used, __float_as_uint(acc[0]));
@@ -542,12 +549,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kProducerWarp)
-    producer(s, p, &tq, &tk);
-  else if (warp == kMmaWarp)
-    mma_issuer(s, p);
-  else if (warp >= kSoftmaxWarp0)
+  if (warp < kSoftmaxWarp0) {
+    regs_dec<kRegsControl>();
+    if (warp == kProducerWarp)
+      producer(s, p, &tq, &tk);
+    else if (warp == kMmaWarp)
+      mma_issuer(s, p);
+  } else {
+    regs_inc<kRegsSoftmax>();
     softmax_group(s, p, (warp - kSoftmaxWarp0) >> 2);
+  }
   __syncwarp();
   tc_fence_before();
   __syncthreads();
@@ -595,8 +606,13 @@ cudaError_t tc_compress_stats(const CompressArgs& a) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = p.n_units < sms ? p.n_units : sms;
+  // the register split assumes the launch allocation it was sized for
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, k_compress_tc);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
   const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(k_compress_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = cudaFuncSetAttribute(k_compress_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps(kKCompressTc, a.stream);
   k_compress_tc<<<grid, kThreads, smem, a.stream>>>(tq, tk, p);
