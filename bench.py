@@ -207,14 +207,17 @@ def source_hash(files):
     return h.hexdigest()[:16]
 
 
-def traffic_for(kernel: str):
-    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if its sources are unchanged."""
+def traffic_for(kernel: str, workload: str):
+    """Per-launch DRAM bytes of `kernel` on `workload` from the committed ncu summary, if its
+    sources are unchanged since the counters were taken (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     try:
         with open(p) as f:
             d = json.load(f)
+        if d.get("workload") != workload:
+            return None
         ent = d.get(kernel)
         if not ent:
             return None
@@ -747,7 +750,7 @@ def main():
     pk, pk_src = peaks()
     dname, (dms, dcnt) = max(prof.items(), key=lambda kv: kv[1][0])
     roofline = roofline_of(dname, dms, dcnt, work, pk, pk_src)
-    roofline["traffic"] = traffic_for(dname)
+    roofline["traffic"] = traffic_for(dname, spec.name + ("+fp8" if fp8 else ""))
     stages = {k: {"ms_per_launch": v[0] / v[1], "launches": v[1], "share": v[0] / sum(x[0] for x in prof.values())}
               for k, v in prof.items()}
     sms = torch.cuda.get_device_properties(local).multi_processor_count

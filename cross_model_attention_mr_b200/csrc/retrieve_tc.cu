@@ -47,8 +47,11 @@ constexpr int kThreads = 576;
 constexpr int kMixThreads = kMixWarps * 32;
 constexpr int kRowsW = 128 / kMixWarps;                  // unit rows per mixer warp
 constexpr int kPieces = 128 * 8 / kMixThreads;           // 16-byte pieces per thread per panel
-constexpr int kQueue = 2;       // entry pairs in flight per mixer thread (its shared-memory ring)
-constexpr int kPages = 12;      // > 2 * kQueue + 2: the fetch cursor never laps the compute cursor
+// entry pairs in flight per mixer thread (its shared-memory ring): an fp8 piece is half the bytes,
+// so the same ring holds twice the pairs
+template <bool F8>
+__host__ __device__ constexpr int queue_of() { return F8 ? 4 : 2; }
+constexpr int kPages = 12;      // > 2 * queue_of<true>() + 2: the fetch cursor never laps the compute cursor
 constexpr int kMaxEntries = 64; // sender heads
 constexpr int kPaceSlack = 4;   // pages a CTA may run ahead of the slowest CTA of its group
 constexpr uint64_t kPaceNs = 100000ull;  // longest hold per page
@@ -86,7 +89,8 @@ struct Params {
 // stored because the map overflowed) and the unit's mixing weights for the panel's sender head.
 struct Entry {
   uint32_t t[2];
-  uint32_t pad[2];
+  uint32_t sc[2];  // fp8 maps: the scale of each 32-row group q of the unit in this panel, as bf16
+                   // (group q in half q % 2 of word q / 2); unused for bf16 maps
   float w[kAcc];
 };
 // One sub-step (n >= 1 entries, panel h of the key block) or a marker (n == 0).
@@ -107,14 +111,16 @@ template <bool F8>
 struct SmemT {
   __nv_bfloat16 x[kAcc][128 * 64];
   __nv_bfloat16 v[kAcc][64 * 128];
-  uint4 ring[kQueue][2][F8 ? kPieces8 : kPieces][kMixThreads];  // [pair slot][entry][piece][mixer thread]
-  float sring[kQueue][2][F8 ? kMixThreads : 1];                  // fp8: each entry's piece scale
+  uint4 ring[queue_of<F8>()][2][F8 ? kPieces8 : kPieces][kMixThreads];  // [pair slot][entry][piece][mixer thread]
   Page page[kPages];
   uint64_t plan_full[kPages], plan_empty[kPages];
   uint64_t x_full, x_empty, v_full, v_empty, o_full, o_empty, mma_done;
   uint32_t tmem_base;
   int abort;
 };
+
+static_assert(sizeof(SmemT<false>) + 1024 <= 232448 && sizeof(SmemT<true>) + 1024 <= 232448,
+              "shared memory of one CTA (plus alignment slack) must fit the 227 KB opt-in limit");
 
 struct Unit {
   int rb, hg, rg, I0, I1, Jmax;
@@ -343,6 +349,25 @@ __device__ void planner(SmemT<F8>& s, const Params& p) {
             }
 #pragma unroll
             for (int g = 0; g < kAcc; ++g) e.w[g] = wv[hs][g];
+            if (F8) {
+              // the scales of the unit's four 32-row groups in panel h (rows 32 q .. of query block
+              // I0 at block 128; two groups of I0 and two of I1 at block 64), rounded to bf16: the
+              // relative error 2^-9 is small beside the e4m3 step of the values they scale
+              uint32_t hb[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int pt = p.B == 128 ? 0 : q >> 1;
+                const int rg = p.B == 128 ? q : q & 1;
+                const uint32_t t = e.t[pt];
+                const float sc = t != kNone ? __ldg(p.tile_scale + (size_t)t * fp8_scales_per_tile(p.B) +
+                                                    rg * (p.B / 64) + (p.B == 128 ? h : 0))
+                                            : 0.f;
+                const __nv_bfloat16 b = __float2bfloat16_rn(sc);
+                hb[q] = *reinterpret_cast<const uint16_t*>(&b);
+              }
+              e.sc[0] = hb[0] | (hb[1] << 16);
+              e.sc[1] = hb[2] | (hb[3] << 16);
+            }
           }
           if (lane == 0) {
             const uint32_t n = (uint32_t)__popcll((long long)uni);
@@ -540,18 +565,10 @@ __device__ void mma_issuer(SmemT<F8>& s, const Params& p, const CUtensorMap* tma
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ float lds32f(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
 }
 // A stored word holds the e4m3 codes of keys (0, 2, 1, 3) of a group of four, all non-negative.
 // Placing a code's 7 bits at bits 7..13 of a half gives exactly its value times 2^-8 (the exponent
@@ -585,12 +602,10 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
   const uint32_t tile_bytes = (uint32_t)(p.B * p.B * 2);
   const char* vals = reinterpret_cast<const char*>(p.vals);
   // fp8 maps: thread (w, l) owns row rowb8 = 8 w + l / 4 of the unit and the 16-key piece l % 4 of
-  // each 64-byte panel row, and fetches the scale of the 32-row x 64-key piece it falls in
+  // each 64-byte panel row; the scale of the 32-row x 64-key piece it falls in comes with the page entry
   const uint32_t rowb8 = (uint32_t)(kRowsW * warp + (lane >> 2));
   const uint32_t trow8 = p.B == 64 ? (rowb8 & 63u) : rowb8;
   const uint32_t my_off8 = trow8 * 64u + (uint32_t)(lane & 3) * 16u;
-  const uint32_t sc_row8 = (trow8 >> 5) * (uint32_t)(p.B / 64);
-  const uint32_t nsc = (uint32_t)fp8_scales_per_tile(p.B);
   const char* vals8 = reinterpret_cast<const char*>(p.vals8);
   const uint32_t tbase = s.tmem_base;
   const int tw = warp & 3;  // Tensor Memory lane quadrant of this warp
@@ -641,8 +656,7 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
   const uint32_t ring0 = smem_u32(&s.ring[0][0][0][threadIdx.x]);
   constexpr int kPc = F8 ? kPieces8 : kPieces;
   constexpr uint32_t kPiece = kMixThreads * 16u, kEntry = kPc * kPiece, kSlot = 2u * kEntry;
-  const uint32_t sring0 = smem_u32(&s.sring[0][0][F8 ? threadIdx.x : 0]);
-  constexpr uint32_t kSEntry = kMixThreads * 4u, kSSlot = 2u * kSEntry;
+  constexpr int kQueue = queue_of<F8>();
   auto fetch = [&](uint32_t slot) -> bool {
     bool good = true;
     if (!f_done && ef == nf) good = fetch_seek(pf + 1);
@@ -654,7 +668,6 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
         const uint64_t t = tt[j];
         cp_async16(ring0 + slot * kSlot + j * kEntry,
                    vals8 + (t * (uint64_t)(p.B * p.B) + hf * 64u * (uint32_t)p.B + my_off8));
-        cp_async4(sring0 + slot * kSSlot + j * kSEntry, p.tile_scale + (t * nsc + sc_row8 + hf));
       }
       ++ef;
     } else if (good && !f_done) {
@@ -689,8 +702,9 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
     }
 
   // fp8 entry: acch[g] += (W[r_g, s] * scale * 2^14) * (the thread's 16 e4m3 values)
-  auto mix_entry8 = [&](const Entry& E, uint32_t data, uint32_t sdata) {
-    const float sc = lds32f(sdata) * (kF8Pre * kF8Decode);
+  auto mix_entry8 = [&](const Entry& E, uint32_t data) {
+    const uint32_t scw = E.sc[rowb8 >> 6];
+    const float sc = __uint_as_float((rowb8 & 32u) ? (scw & 0xffff0000u) : (scw << 16)) * (kF8Pre * kF8Decode);
     __half2 w2[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) w2[g] = __float2half2_rn(E.w[g] * sc);
@@ -851,7 +865,7 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
       const Entry& E = cpg->e[2 * ec + j];
       if (E.t[half] != kNone) {
         if (F8)
-          mix_entry8(E, data + j * kEntry, sring0 + slot * kSSlot + j * kSEntry);
+          mix_entry8(E, data + j * kEntry);
         else
           mix_entry(E, data + j * kEntry);
       }
