@@ -246,7 +246,7 @@ __device__ void softmax_group(Smem& s, const Params& p, int w) {
       // their latency hides behind the MMA
       float kbo[4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) kbo[c] = kb_offset(p.bias, h, 128 * T + 32 * c);
+      for (int cc = 0; cc < 4; ++cc) kbo[cc] = kb_offset(p.bias, h, 128 * T + 32 * cc);
       if (!mbar_wait(&s.s_full[w], nb & 1, &s.abort, kTimeoutNs)) {
         // Leave the tile loop but still pass the epilogue's barriers of this unit: the other
         // warpgroup's bounded waits see the abort flag and meet us there.

@@ -291,8 +291,12 @@ def test_full_size_sampled(mr, n):
     lay = draw_layers(spec)[0]
     m, O, st = run_layer(mr, spec, lay)
     assert st == mr.MR_OK
-    stats = compare_compress(spec, lay, m, _sample_units(spec, 4, n), n_tiles=6)
-    rows = np.array([0, 5, spec.L // 2 + 17, spec.L - 1])
+    stats = compare_compress(spec, lay, m, _sample_units(spec, 12, n), n_tiles=12)
+    # rows at both ends, at 128-row block edges and inside blocks across the whole length
+    L = spec.L
+    rng = np.random.default_rng(100 + n)
+    rows = np.unique(np.concatenate([[0, 5, 127, 128, L // 4 + 3, L // 2 + 17, L // 2 + 64, 3 * L // 4 + 101,
+                                      L - 129, L - 128, L - 2, L - 1], rng.integers(0, L, size=6)]))
     rel = compare_retrieve(spec, lay, m, O, rows)
     print(spec.name, stats, rel)
 
