@@ -32,6 +32,7 @@ constexpr int kSoftmaxWarp0 = 4;
 constexpr int kKStages = 3;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLog2Fp8Max = 8.807354922057604f;  // log2(448), 448 = largest e4m3 value
 
 struct Params {
   int H, L, B, nqb, nkw, n_rb, n_units;
@@ -300,6 +301,43 @@ __device__ void emit_group(Smem& s, const Params& p, int w) {
           if (lane == 0) mbar_arrive(&s.s_empty[w]);
         }
         if (!((row_mask >> hh) & 1u)) continue;  // warp-uniform
+        if (F8 && !special) {
+          // fp8, bias constant per 32 keys: the piece maximum comes from the raw logits (a > 0),
+          // so each value is produced already scaled, P * 448 / max = 2^(x + log2 448 - max x),
+          // by one FMA and one exponential
+          float ob[2], mxl = -INFINITY;
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            ob[cc] = kb_offset(p.bias, h, j_tile + 64 * hh + 32 * cc) - lse2;
+            float m = __uint_as_float(raw[cc][0]);
+#pragma unroll
+            for (int t = 1; t < 32; ++t) m = fmaxf(m, __uint_as_float(raw[cc][t]));
+            mxl = fmaxf(mxl, fmaf(m, p.a, ob[cc]));
+          }
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) mxl = fmaxf(mxl, __shfl_xor_sync(0xffffffffu, mxl, o));
+          sc[hh] = ex2_approx(mxl) / kFp8Max;
+          const float shift = kLog2Fp8Max - mxl;
+          char* dst = stage + 2048 * hh + lane * 64;
+#pragma unroll
+          for (int c16 = 0; c16 < 4; ++c16) {
+            const int cc = c16 >> 1;
+            const float o = ob[cc] + shift;
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int x = 16 * (c16 & 1) + 4 * e;
+              float q[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) q[u] = ex2_approx(fmaf(__uint_as_float(raw[cc][x + u]), p.a, o));
+              const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(q[0], q[1]), __NV_SATFINITE, __NV_E4M3);
+              const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(q[2], q[3]), __NV_SATFINITE, __NV_E4M3);
+              pk[e] = __byte_perm(lo, hi, 0x5140);  // bytes of keys (0, 2, 1, 3)
+            }
+            *reinterpret_cast<uint4*>(dst + 16 * c16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+          continue;
+        }
         float pr[64];
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
