@@ -25,7 +25,16 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 384;
+// Warpgroup 0: TMA producer warp, MMA warp, two idle warps; warpgroups 1..kWG: emitting
+// warpgroups, which take the unit's needed tiles in turn.  Three of them put three emitting warps
+// on every SM sub-partition (the kernel is bound by their latency); warpgroup 0 drops to 56
+// registers so they can rise to 152 each: 56 + 3 x 152 = 4 x 128, the launch allocation.
+constexpr int kWG = 3;
+constexpr int kThreads = 128 * (kWG + 1);
+constexpr int kLaunchRegs = 128;
+constexpr int kRegsControl = 56;
+constexpr int kRegsEmit = 152;
+static_assert(kRegsControl + kWG * kRegsEmit == (kWG + 1) * kLaunchRegs, "register split");
 constexpr int kProducerWarp = 0;
 constexpr int kMmaWarp = 1;
 constexpr int kSoftmaxWarp0 = 4;
@@ -53,14 +62,16 @@ struct Params {
 struct Smem {
   __nv_bfloat16 q[2][128 * 64];
   __nv_bfloat16 k[kKStages][2][128 * 64];
-  __nv_bfloat16 stage[2][128 * 128];  // per warpgroup: 4 warps x (2 key halves x 32 rows x 128 B)
+  __nv_bfloat16 stage[kWG][128 * 128];  // per warpgroup: 4 warps x (2 key halves x 32 rows x 128 B)
   uint64_t q_full, q_empty;
   uint64_t k_full[kKStages], k_empty[kKStages];
-  uint64_t s_full[2], s_empty[2];
+  uint64_t s_full[kWG], s_empty[kWG];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
 };
+
+static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory (plus alignment slack) must fit the 227 KB opt-in limit");
 
 __device__ __forceinline__ void fail(Smem& s, const Params& p, uint32_t detail) {
   set_status(p.ws, MR_ERR_TIMEOUT, detail);
@@ -191,7 +202,7 @@ __device__ void mma_issuer(Smem& s, const Params& p) {
   if ((threadIdx.x & 31) != 0) return;
   const uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
   const uint32_t tbase = s.tmem_base;
-  uint32_t nk = 0, nu = 0, nb[2] = {0, 0};
+  uint32_t nk = 0, nu = 0, nb[kWG] = {};
   bool ok = true;
   for (int k = blockIdx.x; k < p.n_units && ok; k += gridDim.x, ++nu) {
     int h, rb;
@@ -206,7 +217,7 @@ __device__ void mma_issuer(Smem& s, const Params& p) {
     for (int T = 0; T <= rb; ++T) {
       int64_t tpos[4];
       if (!uc.pieces(p, T, tpos)) continue;
-      const int st = (int)(nk % kKStages), b = n_local & 1;
+      const int st = (int)(nk % kKStages), b = n_local % kWG;
       if (!mbar_wait(&s.k_full[st], (nk / kKStages) & 1, &s.abort, kTimeoutNs) ||
           (nb[b] > 0 && !mbar_wait(&s.s_empty[b], (nb[b] - 1) & 1, &s.abort, kTimeoutNs))) {
         fail(s, p, 0x512);
@@ -269,7 +280,7 @@ __device__ void emit_group(Smem& s, const Params& p, int w) {
       int64_t tpos[4];
       const uint32_t pieces = uc.pieces(p, T, tpos);
       if (!pieces) continue;
-      const int mine = n_local++ & 1;
+      const int mine = n_local++ % kWG;
       if (mine != w) continue;
       if (!mbar_wait(&s.s_full[w], nb & 1, &s.abort, kTimeoutNs)) {
         fail(s, p, 0x521);
@@ -446,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.k_full[i], 1);
       mbar_init(&s.k_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kWG; ++i) {
       mbar_init(&s.s_full[i], 1);
       mbar_init(&s.s_empty[i], 4);
     }
@@ -455,23 +466,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(&s.tmem_base, 256);
+    tmem_alloc(&s.tmem_base, 512);  // kWG S buffers of 128 columns (allocations are powers of two)
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kProducerWarp)
-    producer(s, p, &tq, &tk);
-  else if (warp == kMmaWarp)
-    mma_issuer(s, p);
-  else if (warp >= kSoftmaxWarp0)
+  // every warp of warpgroup 0 gives its registers back before any role starts: the emitting
+  // warpgroups' increase waits for them
+  if (warp < kSoftmaxWarp0) {
+    regs_dec<kRegsControl>();
+    if (warp == kProducerWarp)
+      producer(s, p, &tq, &tk);
+    else if (warp == kMmaWarp)
+      mma_issuer(s, p);
+  } else {
+    regs_inc<kRegsEmit>();
     emit_group<F8>(s, p, (warp - kSoftmaxWarp0) >> 2);
+  }
   __syncwarp();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(s.tmem_base, 256);
+  if (warp == kMmaWarp) tmem_dealloc(s.tmem_base, 512);
 }
 
 }  // namespace
@@ -510,7 +527,13 @@ cudaError_t tc_emit(const CompressArgs& a) {
   const size_t smem = sizeof(Smem) + 1024;
   const bool f8 = a.map.val_dtype == MR_FP8_E4M3;
   auto kern = f8 ? k_emit_tc<true> : k_emit_tc<false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // the register split assumes the launch allocation it was sized for; anything else could leave
+  // an increase waiting for registers that do not exist
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps(kKEmitTc, a.stream);
   kern<<<grid, kThreads, smem, a.stream>>>(tq, tk, p);
