@@ -53,6 +53,24 @@ def test_library_variant_matches_environment(mr):
     assert mr.LIB.mr_checked_build() == (1 if os.environ.get("MR_LIBRARY") == "checked" else 0)
 
 
+def test_bench_traffic_is_tied_to_its_workload_and_sources():
+    """The bench line's DRAM traffic comes from the committed capture only for the workload it was
+    scaled to, and only while the kernel sources it was taken on are unchanged."""
+    import json
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    d = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    wl = d["workload"]
+    for kernel in ("mr_compress_tc", "mr_emit_tc", "mr_retrieve_tc"):
+        ent = d[kernel]
+        fresh = bench.source_hash(ent["sources"]) == ent["source_hash"]
+        got = bench.traffic_for(kernel, wl)
+        assert (got == ent["bytes_per_launch"]) if fresh else got is None
+        assert bench.traffic_for(kernel, wl + "+fp8") is None
+        assert bench.traffic_for(kernel, "L8192_32to64_d128_bf16_B128") is None
+
+
 def test_status_strings(mr):
     for code in range(8):
         s = mr.LIB.mr_status_string(code)

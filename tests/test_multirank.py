@@ -95,6 +95,22 @@ def _synthetic_map(mr, nnz, capacity, seed, dtype=None):
     return m
 
 
+def test_map_copy_between_devices_keeps_every_array():
+    """Map.to: the copy a receiving rank makes to move a received map onto its GPU (here host to
+    host) keeps capacity, flags and every array bit for bit."""
+    from cross_model_attention_mr_b200 import mr
+    for dt in (None, mr.MR_FP8_E4M3):
+        src = _synthetic_map(mr, 29, 32, seed=7, dtype=dt)
+        dst = src.to("cpu")
+        assert dst is not src and dst.capacity == src.capacity and dst.c.capacity_tiles == src.c.capacity_tiles
+        assert dst.dtype == src.dtype and dst.c.renormalised == src.c.renormalised
+        for name in ("row_ptr", "col_idx", "vals", "kept_mass", "kept_bits", "nnz", "tile_scale"):
+            a, b = getattr(src, name), getattr(dst, name)
+            assert (a is None) == (b is None)
+            if a is not None:
+                assert a.data_ptr() != b.data_ptr() and torch.equal(a, b), name
+
+
 def _map_rank_main(rank, world, port, out):
     sys.path.insert(0, ROOT)
     os.environ["MASTER_ADDR"] = "127.0.0.1"
