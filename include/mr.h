@@ -426,10 +426,12 @@ mr_status mr_gather_probe(const mr_bsr* map, int readers, int ring_slots, void* 
 
 /*
  * Failure-path test hook (not part of the method; process-wide, for tests).  Sets the limit of the
- * tensor-core dense kernel's protocol waits to wait_ns (0 = the default 2 s) and, with
- * skip_arrive = 1, makes its softmax warpgroup withhold its first "P ready" arrive, so the MMA
- * warp's wait runs out: the call records MR_ERR_TIMEOUT (detail 0x913) in the workspace's status
- * word, drains its copies and MMAs, frees Tensor Memory and returns, leaving the context usable.
+ * tensor-core dense kernel's protocol waits to wait_ns (0 = the default 2 s; its softmax
+ * warpgroups wait twice as long, so the wait nearest a stall reports it) and, with
+ * skip_arrive = 1, makes the softmax warpgroup of each CTA's first query tile withhold its first
+ * "P ready" arrive, so the MMA warp's wait runs out: the call records MR_ERR_TIMEOUT (detail
+ * 0x913) in the workspace's status word, drains its copies and MMAs, frees Tensor Memory and
+ * returns, leaving the context usable.
  * mr_debug_set(0, 0) restores normal operation.  No GPU fault is involved.
  */
 mr_status mr_debug_set(uint64_t wait_ns, int skip_arrive);
