@@ -40,10 +40,7 @@ using namespace sm100;
 // thread at 96 registers: enough for 4 x 16 fp32 accumulators (2 pieces per thread) with the
 // paired FMA as a compiler builtin.  Measured against 8 mixer warps with 4 pieces each (168
 // registers): 4 mixer warps per sub-partition hide more latency, 5% faster at 32K tokens.
-constexpr int kMixWarps = 16;
-constexpr int kPlanWarp = 16;
-constexpr int kMmaWarp = 17;
-constexpr int kThreads = 576;
+constexpr int kMixWarps = 16;  // CUDA-core mixing path (the tensor-core one runs 8, see Roles)
 constexpr int kMixThreads = kMixWarps * 32;
 constexpr int kRowsW = 128 / kMixWarps;                  // unit rows per mixer warp
 constexpr int kPieces = 128 * 8 / kMixThreads;           // 16-byte pieces per thread per panel
@@ -112,6 +109,7 @@ struct SmemT {
   __nv_bfloat16 x[kAcc][128 * 64];
   __nv_bfloat16 v[kAcc][64 * 128];
   uint4 ring[queue_of<F8>()][2][F8 ? kPieces8 : kPieces][kMixThreads];  // [pair slot][entry][piece][mixer thread]
+  uint4 xpad[8][32];  // tensor-core mixing: a 512-byte scratch per mixer warp for the zero rows of its products
   Page page[kPages];
   uint64_t plan_full[kPages], plan_empty[kPages];
   uint64_t x_full, x_empty, v_full, v_empty, o_full, o_empty, mma_done;
@@ -236,7 +234,7 @@ __device__ void planner(SmemT<F8>& s, const Params& p) {
   auto claim = [&]() -> Page* {
     bool good = true;
     if (lane == 0 && np >= (uint32_t)kPages &&
-        !mbar_wait_sleep(&s.plan_empty[np % kPages], ((np / kPages) - 1) & 1, &s.abort, kTimeoutNs, 256)) {
+        !mbar_wait_hint(&s.plan_empty[np % kPages], ((np / kPages) - 1) & 1, &s.abort, kTimeoutNs)) {
       fail(s, p, 0x101);
       good = false;
     }
@@ -487,7 +485,7 @@ __device__ void mma_issuer(SmemT<F8>& s, const Params& p, const CUtensorMap* tma
   const int nu = units_of_cta(p);
   for (; nunit < nu && ok; ++nunit) {
     const Unit u = unit_at(p, nunit);
-    if (lane == 0 && nunit > 0 && !mbar_wait_sleep(&s.o_empty, (nunit - 1) & 1, &s.abort, kTimeoutNs, 64)) {
+    if (lane == 0 && nunit > 0 && !mbar_wait_hint(&s.o_empty, (nunit - 1) & 1, &s.abort, kTimeoutNs)) {
       fail(s, p, 0x201);
       ok = false;
     }
@@ -500,8 +498,8 @@ __device__ void mma_issuer(SmemT<F8>& s, const Params& p, const CUtensorMap* tma
       if ((m0 | m1) == 0) continue;
       for (int h = 0; h < nparts && ok; ++h) {
         if (lane == 0) {
-          if (!mbar_wait_sleep(&s.x_full, nsub & 1, &s.abort, kTimeoutNs, 64) ||
-              !mbar_wait_sleep(&s.v_full, nsub & 1, &s.abort, kTimeoutNs, 64)) {
+          if (!mbar_wait_hint(&s.x_full, nsub & 1, &s.abort, kTimeoutNs) ||
+              !mbar_wait_hint(&s.v_full, nsub & 1, &s.abort, kTimeoutNs)) {
             fail(s, p, 0x202);
             ok = false;
           } else {
@@ -529,7 +527,7 @@ __device__ void mma_issuer(SmemT<F8>& s, const Params& p, const CUtensorMap* tma
         // the next sub-step's V, once these MMAs have read the buffer
         if (vw.next(p)) {
           if (lane == 0) {
-            if (!mbar_wait_sleep(&s.v_empty, (nsub - 1) & 1, &s.abort, kTimeoutNs, 64)) {
+            if (!mbar_wait_hint(&s.v_empty, (nsub - 1) & 1, &s.abort, kTimeoutNs)) {
               fail(s, p, 0x203);
               ok = false;
             } else {
@@ -582,6 +580,51 @@ __device__ __forceinline__ __half2 e4m3_pair23(uint32_t w) {
   const uint32_t h = (w >> 1) & 0x3F803F80u;
   return *reinterpret_cast<const __half2*>(&h);
 }
+// Four 8x8 b16 matrices from shared memory, transposed (thread t gets rows 2 (t % 4), + 1 of
+// column t / 4 of each); lanes 8 m .. 8 m + 7 give the row addresses of matrix m.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+// D (16 x 8, fp32) += A (16 x 16, bf16, row-major) * B (16 x 8, bf16, column-major), register operands.
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+               "{%0, %1, %2, %3};"
+               : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// As cp_async16, issued only where `pred` holds (no branch).
+__device__ __forceinline__ void cp_async16_if(uint32_t dst, const void* src, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %2, 0;\n\t@p cp.async.cg.shared.global [%0], [%1], 16;\n\t}" ::"r"(dst),
+      "l"(src), "r"((uint32_t)pred)
+      : "memory");
+}
+template <int N>
+struct Int {
+  static constexpr int value = N;
+};
+// D (16 x 8, fp32) = A (16 x 16, bf16; rows 8 .. 15 zero) * B (16 x 8, bf16): the first k-step of a row.
+__device__ __forceinline__ void mma_16816_z(float (&c)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %5}, {%7, %8}, "
+               "{%9, %9, %9, %9};"
+               : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+               : "r"(a0), "r"(0u), "r"(a2), "r"(b0), "r"(b1), "f"(0.f));
+}
+// Four 8x8 b16 matrices to shared memory in the MMA accumulator layout (thread t holds row t / 4,
+// columns 2 (t % 4), + 1 of each); lanes 8 m .. 8 m + 7 give the row addresses of matrix m.
+__device__ __forceinline__ void stsm_x4(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(r0), "r"(r1), "r"(r2),
+               "r"(r3)
+               : "memory");
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&b2);
+}
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
@@ -593,7 +636,9 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 // l % 8 of the 128-byte-swizzled
 // panel row: eight consecutive keys 8 * ((l % 8) ^ (a_k % 8)).  X is written with the same
 // swizzle, so the thread writes its chunks back to the positions it read them from.
-template <int G, bool F8>
+// MM: mix on the tensor core with register operands (bf16 maps, block 128, at most 32 sender heads,
+// 4 receiver heads of one request group); otherwise in fp32 / half FMAs on the CUDA cores.
+template <int G, bool F8, bool MM>
 __device__ void mixers(SmemT<F8>& s, const Params& p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int half = p.B == 64 ? (warp / (kMixWarps / 2)) : 0;  // 64-key blocks: which of the unit's two query blocks
@@ -621,7 +666,7 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
   int nunit = 0;
 
   auto wait_page = [&](uint32_t pg) -> bool {
-    return mbar_wait(&s.plan_full[pg % kPages], (pg / kPages) & 1, &s.abort, kTimeoutNs);
+    return mbar_wait_hint(&s.plan_full[pg % kPages], (pg / kPages) & 1, &s.abort, kTimeoutNs);
   };
   auto release_page = [&](uint32_t pg) {
     __syncwarp();
@@ -746,7 +791,7 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
 
   // X of one sub-step, once the previous sub-step's MMAs have read the buffer
   auto hand_x = [&]() -> bool {
-    if (nsub > 0 && !mbar_wait(&s.x_empty, (nsub - 1) & 1, &s.abort, kTimeoutNs)) return false;
+    if (nsub > 0 && !mbar_wait_hint(&s.x_empty, (nsub - 1) & 1, &s.abort, kTimeoutNs)) return false;
 #pragma unroll
     for (int g = 0; g < (F8 ? G : 0); ++g) {
 #pragma unroll
@@ -788,7 +833,7 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
   };
   // the unit's accumulators -> bf16 -> O (warp w stores accumulators w / 4 + 2 i of its 32 rows)
   auto epilogue = [&](bool any) -> bool {
-    if (!mbar_wait(&s.o_full, nunit & 1, &s.abort, kTimeoutNs)) return false;
+    if (!mbar_wait_hint(&s.o_full, nunit & 1, &s.abort, kTimeoutNs)) return false;
     tc_fence_after();
     const Unit u = unit_at(p, nunit);
     const int row = 32 * tw + lane;
@@ -797,7 +842,7 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
     const bool row_out = i < p.L && qblk >= p.qb0 && qblk < p.qb1;  // rows outside the range stay as they are
     const float osc = F8 ? 1.f / kF8Pre : 1.f;                       // fp8 maps were mixed x 2^14
 #pragma unroll 1
-    for (int a = warp >> 2; a < G * p.R; a += kMixWarps / 4) {
+    for (int a = warp >> 2; a < G * p.R; a += (MM ? 8 : kMixWarps) / 4) {
       const bool valid = acc_valid(p, u, G, a);
       const int r = u.hg * G + a / p.R, q = u.rg * p.R + a % p.R;
       __nv_bfloat16* orow = p.O + (((size_t)q * p.H_r + r) * p.L + i) * 128;
@@ -852,6 +897,219 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
     }
   };
 
+  if (MM) {
+    // ---- head mixing as a tensor-core contraction over sender heads ---------------------------
+    // X_g[i, j] = sum_s W[g, s] A_s[i, j] is, for each unit row i, a product of the page's weights
+    // (A operand: 16 rows, the first G of them receiver heads; 16 sender heads per k-step) and the
+    // sender heads' values in that row (B operand: 16 heads x 8 keys per n-tile, through a
+    // transposed matrix load), accumulated in fp32 registers: no Tensor Memory (all of it holds the
+    // Ã·V accumulators) and no per-thread accumulator arrays.  8 mixer warps; warp w owns unit rows
+    // 16 w .. 16 w + 15.  A step is one row and one k-step: the row's 128 bytes in each of 16
+    // sender heads, copied by the warp into a private 2 KB slot of a 4-deep ring, so the warp waits
+    // on its own copies only.  Head e's row sits at e * 128 with the map's physical chunk q at
+    // q ^ (e % 8), so the eight rows of each transposed load hit eight different bank groups.
+    constexpr uint32_t kD = 4, kRows = 16;
+    static_assert(sizeof(s.ring) == 8 * kD * 2048, "8 warps x kD slots of 2 KB");
+    static_assert(!MM || G == 4, "the first four rows of the product are the receiver heads");
+    char* wring_g = reinterpret_cast<char*>(&s.ring[0][0][0][0]) + (uint32_t)warp * (kD * 2048u);
+    const uint32_t wring = smem_u32(wring_g);
+    for (uint32_t off = (uint32_t)lane * 16u; off < kD * 2048u; off += 512u)
+      *reinterpret_cast<uint4*>(wring_g + off) = make_uint4(0u, 0u, 0u, 0u);  // unlisted heads: weight 0, finite values
+    __syncwarp();
+    const uint32_t q = (uint32_t)lane & 7u, lh = (uint32_t)lane >> 3;
+    // copies: lane (lh, q) moves chunk q of heads 4 jj + lh (jj < 4); slot offsets for even and odd
+    // jj, + 1024 for jj >= 2
+    const uint32_t dst_even = lh * 128u + ((q ^ lh) << 4), dst_odd = 512u + lh * 128u + ((q ^ (4u + lh)) << 4);
+    // transposed loads: lane 8 m + r gives row r of matrix m, i.e. head 8 (m % 2) + r and logical
+    // chunk 2 i + m / 2 of the row, stored at (2 i + m / 2) ^ (row % 8) ^ r
+    const uint32_t ld_row = (8u * (lh & 1u) + q) * 128u, ld_z = (lh >> 1) ^ q;
+    // matrix stores of a finished row: lane 8 m + r gives row r of n-tile 4 k + m.  Rows r < 4 are
+    // the receiver heads' X rows; rows 4..7 of the product are zero and go to a scratch line of this
+    // warp, at the other half of the bank groups
+    const bool st_real = q < 4u;
+    const uint32_t st_base = st_real ? smem_u32(&s.x[q & 3u][0]) : smem_u32(&s.xpad[warp][0]) + (q - 4u) * 128u;
+    const uint32_t st_rowmask = st_real ? 0xffffffffu : 0u;
+    const uint32_t st_u0 = (lh << 4) ^ (st_real ? 0u : 64u);
+    auto store_row = [&](uint32_t row, const uint32_t (&w)[8]) {
+      const uint32_t R = kRows * (uint32_t)warp + row;
+      const uint32_t base = st_base + ((R * 128u) & st_rowmask);
+      const uint32_t u = st_u0 ^ ((R & 7u) << 4);
+      stsm_x4(base | u, w[0], w[1], w[2], w[3]);
+      stsm_x4(base | (u ^ 64u), w[4], w[5], w[6], w[7]);
+    };
+
+    // fetch cursor: page, step within it (row = step >> f_sh, k-step = step & f_sh), the lane's tiles
+    uint32_t f_pg = 0, f_s = 0, f_steps = 0, f_sh = 0;
+    bool f_end = false;
+    const char* f_src = vals;  // chunk q of the warp's first row in the page's panel of tile 0
+    uint32_t tl0[4], tl1[4];   // tiles of heads 4 jj + lh and 16 + 4 jj + lh (kNone: no copy)
+    auto f_seek = [&](uint32_t from) -> bool {
+      for (uint32_t pg = from;; ++pg) {
+        if (!wait_page(pg)) return false;
+        const Page* P = &s.page[pg % kPages];
+        const uint32_t n = P->n;
+        if (n > 0) {
+          f_pg = pg;
+          f_s = 0;
+          f_sh = n > 16u ? 1u : 0u;
+          f_steps = kRows << f_sh;
+          f_src = vals + (P->h * 16384u + (uint32_t)warp * (kRows * 128u) + q * 16u);
+#pragma unroll
+          for (uint32_t jj = 0; jj < 4; ++jj) {
+            const uint32_t e0 = 4u * jj + lh, e1 = 16u + e0;
+            tl0[jj] = e0 < n ? P->e[e0].t[0] : kNone;
+            tl1[jj] = e1 < n ? P->e[e1].t[0] : kNone;
+          }
+          return true;
+        }
+        if (P->flags & kEnd) {
+          f_end = true;
+          return true;
+        }
+      }
+    };
+    // copy the next step into `slot`: one cp.async group per step, empty at the end
+    auto fetch_step = [&](uint32_t slot) -> bool {
+      bool ok = true;
+      if (!f_end && f_s == f_steps) ok = f_seek(f_pg + 1);
+      if (ok && !f_end) {
+        const uint32_t kt = f_s & f_sh;
+        const char* src = f_src + (f_s >> f_sh) * 128u;
+        const uint32_t d = wring + slot * 2048u;
+#pragma unroll
+        for (uint32_t jj = 0; jj < 4; ++jj) {
+          const uint32_t t = kt ? tl1[jj] : tl0[jj];
+          cp_async16_if(d + ((jj & 1u) ? dst_odd : dst_even) + (jj >> 1) * 1024u, src + (uint64_t)t * 32768u, t != kNone);
+        }
+        ++f_s;
+      }
+      cp_async_commit();
+      return ok;
+    };
+    // A fragments of the compute page: receiver lane / 4 (zero beyond G), heads 16 kt + 2 (lane % 4)
+    // + {0, 1} (first register) and + 8 + {0, 1} (second); rows 8 .. 15 of A are zero
+    uint32_t afr[2][2];
+    uint32_t c_nkt = 1;
+    auto build_a = [&]() {
+      const uint32_t n = cpg->n;
+      c_nkt = n > 16u ? 2u : 1u;
+      const int g = lane >> 2;
+#pragma unroll
+      for (int kt = 0; kt < 2; ++kt)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint32_t e0 = 16u * kt + 8u * hh + 2u * ((uint32_t)lane & 3u);
+          float w0 = 0.f, w1 = 0.f;
+          if (g < G) {
+            if (e0 < n && cpg->e[e0].t[0] != kNone) w0 = cpg->e[e0].w[g];
+            if (e0 + 1u < n && cpg->e[e0 + 1u].t[0] != kNone) w1 = cpg->e[e0 + 1u].w[g];
+          }
+          afr[kt][hh] = pack_bf16x2(w0, w1);
+        }
+    };
+    bool stop = false;
+    bool good = f_seek(0) && compute_seek(stop);
+    if (good && !stop) build_a();
+    for (uint32_t u = 0; u < kD; ++u)
+      if (good && !stop) good = fetch_step(u);
+    uint32_t slot = 0;
+    // copy step (row, KT) of the compute page into `slot` (the fetch cursor's tiles are that page's)
+    auto fetch_static = [&](uint32_t slot_, uint32_t row, auto KT) {
+      const char* src = f_src + row * 128u;
+      const uint32_t d = wring + slot_ * 2048u;
+#pragma unroll
+      for (uint32_t jj = 0; jj < 4; ++jj) {
+        const uint32_t t = decltype(KT)::value ? tl1[jj] : tl0[jj];
+        cp_async16_if(d + ((jj & 1u) ? dst_odd : dst_even) + (jj >> 1) * 1024u, src + (uint64_t)t * 32768u, t != kNone);
+      }
+      cp_async_commit();
+    };
+    // one k-step of a row: wait for its slot, load it as B fragments, multiply, refill the slot with
+    // the step kD ahead: (row + kD / NKT, KT) of this page, or (TAIL) the next page's first steps
+    auto kstep = [&](uint32_t row, float (&acc)[8][4], auto KT, auto NKT, auto TAIL) {
+      cp_async_wait<kD - 1>();  // this lane's copies of the oldest step have landed
+      __syncwarp();             // ... and every other lane's
+      const uint32_t lrow = wring + slot * 2048u + ld_row;
+      const uint32_t z = (ld_z ^ (row & 7u)) << 4;
+      uint32_t b[4][4];  // [load i][matrix]: n-tiles 2 i and 2 i + 1, heads 0..7 and 8..15 of the k-step
+#pragma unroll
+      for (uint32_t i = 0; i < 4; ++i) ldsm_x4_trans(b[i], lrow | (z ^ (32u * i)));
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        if (decltype(KT)::value == 0)
+          mma_16816_z(acc[nt], afr[0][0], afr[0][1], b[nt >> 1][2 * (nt & 1)], b[nt >> 1][2 * (nt & 1) + 1]);
+        else
+          mma_16816(acc[nt], afr[1][0], 0u, afr[1][1], 0u, b[nt >> 1][2 * (nt & 1)], b[nt >> 1][2 * (nt & 1) + 1]);
+      }
+      __syncwarp();  // every lane's loads of the slot are in the MMAs above before any lane refills it
+      if constexpr (decltype(TAIL)::value) {
+        if (!fetch_step(slot)) good = false;
+      } else {
+        fetch_static(slot, row + kD / decltype(NKT)::value, KT);
+      }
+      slot = (slot + 1u) & (kD - 1u);
+    };
+    // a whole row: its k-steps, then the receivers' X values packed to bf16
+    auto row_x = [&](uint32_t row, uint32_t (&pk)[8], auto NKT, auto TAIL) {
+      float acc[8][4];
+      kstep(row, acc, Int<0>{}, NKT, TAIL);
+      if constexpr (decltype(NKT)::value == 2) kstep(row, acc, Int<1>{}, NKT, TAIL);
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) pk[nt] = pack_bf16x2(acc[nt][0], acc[nt][1]);
+    };
+    // the warp's 16 rows of one sub-step; rows 0..2 are held until X is free.  On entry the fetch
+    // cursor has copied the page's first kD steps; the rest of the page is fetched statically and
+    // the last rows fetch the next page's first kD steps through the cursor.
+    auto sub_step = [&](auto NKT) -> bool {
+      constexpr uint32_t kTail = kRows - kD / decltype(NKT)::value;
+      f_s = f_steps;
+      uint32_t h0[8], h1[8], pk[8];
+      row_x(0, h0, NKT, Int<0>{});
+      row_x(1, h1, NKT, Int<0>{});
+      row_x(2, pk, NKT, Int<0>{});
+      // X is free once the previous sub-step's MMAs have read it
+      bool ok = true;
+      if (lane == 0 && nsub > 0) ok = mbar_wait_hint(&s.x_empty, (nsub - 1) & 1, &s.abort, kTimeoutNs);
+      if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) return false;
+      store_row(0, h0);
+      store_row(1, h1);
+      store_row(2, pk);
+#pragma unroll 1
+      for (uint32_t row = 3; row < kTail; ++row) {
+        row_x(row, pk, NKT, Int<0>{});
+        store_row(row, pk);
+      }
+#pragma unroll 1
+      for (uint32_t row = kTail; row < kRows; ++row) {
+        row_x(row, pk, NKT, Int<1>{});
+        store_row(row, pk);
+      }
+      return true;
+    };
+    while (good && !stop) {
+      const bool ok = c_nkt == 2 ? sub_step(Int<2>{}) : sub_step(Int<1>{});
+      if (!ok || !good) {
+        good = false;
+        break;
+      }
+      // end of the sub-step: X to the tensor core, release the page, run any markers
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.x_full);
+      ++nsub;
+      release_page(pc);
+      ++pc;
+      if (!compute_seek(stop)) {
+        good = false;
+        break;
+      }
+      if (!stop) build_a();
+    }
+    cp_async_wait<0>();  // no copy may land after the CTA releases its shared memory
+    if (!good) fail(s, p, 0x302);
+    return;
+  }
+
   bool stop = false;
   bool good = fetch_seek(0) && compute_seek(stop);
   for (uint32_t u = 0; u < (uint32_t)kQueue; ++u)
@@ -891,8 +1149,16 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
   if (!good) fail(s, p, 0x301);
 }
 
-template <int G, bool F8>
-__global__ void __launch_bounds__(kThreads, 1) k_retrieve_tc(const __grid_constant__ CUtensorMap tmap_v, Params p) {
+// Mixer warps of an instantiation: 16 on the CUDA-core mixing path, 8 on the tensor-core one.
+template <bool MM>
+struct Roles {
+  static constexpr int kMix = MM ? 8 : kMixWarps;
+  static constexpr int kPlan = kMix, kMma = kMix + 1, kThreadsK = (kMix + 2) * 32;
+};
+
+template <int G, bool F8, bool MM>
+__global__ void __launch_bounds__(Roles<MM>::kThreadsK, 1) k_retrieve_tc(const __grid_constant__ CUtensorMap tmap_v, Params p) {
+  constexpr int kMixWarps = Roles<MM>::kMix, kPlanWarp = Roles<MM>::kPlan, kMmaWarp = Roles<MM>::kMma;
   extern __shared__ unsigned char smem_raw[];
   SmemT<F8>& s = *reinterpret_cast<SmemT<F8>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
   const int warp = threadIdx.x >> 5;
@@ -919,7 +1185,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_retrieve_tc(const __grid_consta
   __syncthreads();
   tc_fence_after();
   if (warp < kMixWarps)
-    mixers<G, F8>(s, p);
+    mixers<G, F8, MM>(s, p);
   else if (warp == kPlanWarp)
     planner<G, F8>(s, p);
   else
@@ -930,18 +1196,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_retrieve_tc(const __grid_consta
   if (warp == kMmaWarp) tmem_dealloc(s.tmem_base, 512);
 }
 
-template <int G, bool F8>
+template <int G, bool F8, bool MM = false>
 cudaError_t launch_g(const RetrieveArgs& a, const Params& p, const CUtensorMap& tm, int grid, cudaStream_t st) {
   const size_t smem = sizeof(SmemT<F8>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(k_retrieve_tc<G, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(k_retrieve_tc<G, F8, MM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps(kKRetrieveTc, st);
-  k_retrieve_tc<G, F8><<<grid, kThreads, smem, st>>>(tm, p);
+  k_retrieve_tc<G, F8, MM><<<grid, Roles<MM>::kThreadsK, smem, st>>>(tm, p);
   return cudaGetLastError();
 }
 
 template <bool F8>
 cudaError_t launch_any(const RetrieveArgs& a, const Params& p, const CUtensorMap& tm, int grid, int G) {
+  // bf16 maps of 128-key blocks with at most 32 sender heads, 4 receiver heads per CTA: mixing
+  // on the tensor core
+  if (!F8 && G == 4 && p.B == 128 && p.H_s <= 32) return launch_g<4, false, true>(a, p, tm, grid, a.stream);
   if (G == 4) return launch_g<4, F8>(a, p, tm, grid, a.stream);
   if (G == 2) return launch_g<2, F8>(a, p, tm, grid, a.stream);
   return launch_g<1, F8>(a, p, tm, grid, a.stream);

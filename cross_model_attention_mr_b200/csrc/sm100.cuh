@@ -65,6 +65,34 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// As mbar_try_wait, with a suspend-time hint: while the phase is incomplete the thread may be
+// suspended inside the instruction, and resumes when the phase completes or about `hint_ns` have
+// passed, so a waiting warp neither polls nor sleeps past the completion.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait built on the hinted try-wait: bounded in the same way (timeout, abort flag), checked
+// once per suspension.
+__device__ __forceinline__ bool mbar_wait_hint(uint64_t* bar, uint32_t parity, const volatile int* abort,
+                                               uint64_t timeout_ns, uint32_t hint_ns = 20000) {
+  if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+  }
+}
+
 // Relaxed gpu-scope accesses for counters that other CTAs poll.
 __device__ __forceinline__ void st_relaxed_gpu(uint32_t* ptr, uint32_t v) {
   asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
