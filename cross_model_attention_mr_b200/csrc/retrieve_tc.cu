@@ -106,7 +106,13 @@ constexpr float kF8Decode = 256.f;  // the integer decode yields value * 2^-8
 
 template <bool F8>
 struct SmemT {
-  __nv_bfloat16 x[kAcc][128 * 64];
+  // X of each accumulator (bf16 MMA operand, 128 rows x 64 keys, 128-byte swizzle).  Each buffer
+  // starts 128 bytes further into the swizzle pattern than the one before, so the same row and
+  // chunk of the receivers' buffers fall in different banks.  The tensor core applies the swizzle
+  // to absolute shared-memory addresses (as TMA does): row r of buffer a has phase (r + a) % 8 and
+  // the descriptor is the plain one (measured: a base offset of a in the descriptor reads wrong data).
+  __nv_bfloat16 x[kAcc][128 * 64 + 64];
+  char x_align[1024 - kAcc * 128 % 1024];  // V on a 1024-byte boundary
   __nv_bfloat16 v[kAcc][64 * 128];
   uint4 ring[queue_of<F8>()][2][F8 ? kPieces8 : kPieces][kMixThreads];  // [pair slot][entry][piece][mixer thread]
   uint4 xpad[8][32];  // tensor-core mixing: a 512-byte scratch per mixer warp for the zero rows of its products
@@ -117,6 +123,8 @@ struct SmemT {
   int abort;
 };
 
+static_assert(offsetof(SmemT<false>, v) % 1024 == 0 && offsetof(SmemT<true>, v) % 1024 == 0,
+              "V is a 128-byte-swizzled TMA destination");
 static_assert(sizeof(SmemT<false>) + 1024 <= 232448 && sizeof(SmemT<true>) + 1024 <= 232448,
               "shared memory of one CTA (plus alignment slack) must fit the 227 KB opt-in limit");
 
@@ -805,7 +813,7 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
           acch[g][4 * c + e] = __float2half2_rn(0.f);
         }
         const uint32_t lc = 2u * (uint32_t)(lane & 3) + (uint32_t)c;
-        char* xb = reinterpret_cast<char*>(&s.x[g][0]) + rowb8 * 128 + ((lc ^ (rowb8 & 7u)) << 4);
+        char* xb = reinterpret_cast<char*>(&s.x[g][0]) + rowb8 * 128 + ((lc ^ ((rowb8 + g) & 7u)) << 4);
         *reinterpret_cast<uint4*>(xb) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
     }
@@ -821,7 +829,10 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
           pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
           acc[g][4 * k + e] = make_float2(0.f, 0.f);
         }
-        char* xb = reinterpret_cast<char*>(&s.x[g][0]) + (rowb + 4 * k) * 128 + (lane & 7) * 16;
+        // the chunk read from physical position l % 8 of a panel row (phase row % 8) goes to the
+        // same logical chunk of X row `row` (phase (row + g) % 8)
+        const uint32_t row = rowb + 4 * k;
+        char* xb = reinterpret_cast<char*>(&s.x[g][0]) + row * 128 + (((lane & 7) ^ (row & 7u) ^ ((row + g) & 7u)) << 4);
         *reinterpret_cast<uint4*>(xb) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
     }
@@ -909,6 +920,7 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
     // on its own copies only.  Head e's row sits at e * 128 with the map's physical chunk q at
     // q ^ (e % 8), so the eight rows of each transposed load hit eight different bank groups.
     constexpr uint32_t kD = 4, kRows = 16;
+    constexpr uint32_t kHold = 2;  // rows computed before the wait for X (measured: 2 beats 3)
     static_assert(sizeof(s.ring) == 8 * kD * 2048, "8 warps x kD slots of 2 KB");
     static_assert(!MM || G == 4, "the first four rows of the product are the receiver heads");
     char* wring_g = reinterpret_cast<char*>(&s.ring[0][0][0][0]) + (uint32_t)warp * (kD * 2048u);
@@ -924,16 +936,17 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
     // chunk 2 i + m / 2 of the row, stored at (2 i + m / 2) ^ (row % 8) ^ r
     const uint32_t ld_row = (8u * (lh & 1u) + q) * 128u, ld_z = (lh >> 1) ^ q;
     // matrix stores of a finished row: lane 8 m + r gives row r of n-tile 4 k + m.  Rows r < 4 are
-    // the receiver heads' X rows; rows 4..7 of the product are zero and go to a scratch line of this
-    // warp, at the other half of the bank groups
+    // the receiver heads' X rows (swizzle phase (R + r) % 8); rows 4..7 of the product are zero and
+    // go to scratch line r - 4 of this warp at the phases (R + r) % 8 the receivers leave free, so
+    // the eight rows of each matrix fall in eight different bank groups
     const bool st_real = q < 4u;
     const uint32_t st_base = st_real ? smem_u32(&s.x[q & 3u][0]) : smem_u32(&s.xpad[warp][0]) + (q - 4u) * 128u;
     const uint32_t st_rowmask = st_real ? 0xffffffffu : 0u;
-    const uint32_t st_u0 = (lh << 4) ^ (st_real ? 0u : 64u);
+    const uint32_t st_u0 = lh << 4;
     auto store_row = [&](uint32_t row, const uint32_t (&w)[8]) {
       const uint32_t R = kRows * (uint32_t)warp + row;
       const uint32_t base = st_base + ((R * 128u) & st_rowmask);
-      const uint32_t u = st_u0 ^ ((R & 7u) << 4);
+      const uint32_t u = st_u0 ^ (((R + q) & 7u) << 4);
       stsm_x4(base | u, w[0], w[1], w[2], w[3]);
       stsm_x4(base | (u ^ 64u), w[4], w[5], w[6], w[7]);
     };
@@ -1057,25 +1070,24 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) pk[nt] = pack_bf16x2(acc[nt][0], acc[nt][1]);
     };
-    // the warp's 16 rows of one sub-step; rows 0..2 are held until X is free.  On entry the fetch
+    // the warp's 16 rows of one sub-step; rows 0..kHold are held until X is free.  On entry the fetch
     // cursor has copied the page's first kD steps; the rest of the page is fetched statically and
     // the last rows fetch the next page's first kD steps through the cursor.
     auto sub_step = [&](auto NKT) -> bool {
       constexpr uint32_t kTail = kRows - kD / decltype(NKT)::value;
       f_s = f_steps;
-      uint32_t h0[8], h1[8], pk[8];
-      row_x(0, h0, NKT, Int<0>{});
-      row_x(1, h1, NKT, Int<0>{});
-      row_x(2, pk, NKT, Int<0>{});
+      uint32_t held[kHold + 1][8];
+#pragma unroll
+      for (uint32_t r = 0; r <= kHold; ++r) row_x(r, held[r], NKT, Int<0>{});
       // X is free once the previous sub-step's MMAs have read it
       bool ok = true;
       if (lane == 0 && nsub > 0) ok = mbar_wait_hint(&s.x_empty, (nsub - 1) & 1, &s.abort, kTimeoutNs);
       if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) return false;
-      store_row(0, h0);
-      store_row(1, h1);
-      store_row(2, pk);
+#pragma unroll
+      for (uint32_t r = 0; r <= kHold; ++r) store_row(r, held[r]);
+      uint32_t pk[8];
 #pragma unroll 1
-      for (uint32_t row = 3; row < kTail; ++row) {
+      for (uint32_t row = kHold + 1; row < kTail; ++row) {
         row_x(row, pk, NKT, Int<0>{});
         store_row(row, pk);
       }
