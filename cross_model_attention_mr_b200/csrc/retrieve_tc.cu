@@ -48,8 +48,8 @@ constexpr int kPieces = 128 * 8 / kMixThreads;           // 16-byte pieces per t
 // so the same ring holds twice the pairs
 template <bool F8>
 __host__ __device__ constexpr int queue_of() { return F8 ? 4 : 2; }
-constexpr int kPages = 12;      // > 2 * queue_of<true>() + 2: the fetch cursor never laps the compute cursor
 constexpr int kMaxEntries = 64; // sender heads
+constexpr uint32_t kMmSlots = 5;  // tensor-core mixing: 2 KB ring slots per mixer warp
 constexpr int kPaceSlack = 4;   // pages a CTA may run ahead of the slowest CTA of its group
 constexpr uint64_t kPaceNs = 100000ull;  // longest hold per page
 constexpr int kAcc = 4;
@@ -91,9 +91,10 @@ struct Entry {
   float w[kAcc];
 };
 // One sub-step (n >= 1 entries, panel h of the key block) or a marker (n == 0).
-struct Page {
+template <int E>
+struct PageT {
   uint32_t n, h, flags, pad;
-  Entry e[kMaxEntries];
+  Entry e[E];
 };
 constexpr uint32_t kUnitEnd = 1u, kEmptyUnit = 2u, kEnd = 4u;
 
@@ -104,18 +105,24 @@ constexpr int kPieces8 = 1;
 constexpr float kF8Pre = 16384.f;
 constexpr float kF8Decode = 256.f;  // the integer decode yields value * 2^-8
 
-template <bool F8>
+// MM: the tensor-core mixing (bf16 maps, at most 32 sender heads), with its own ring and a smaller
+// page ring (its fetch cursor is at most one page ahead of the compute cursor).
+template <bool F8, bool MM>
 struct SmemT {
+  // CUDA-core mixing: > 2 * queue_of<true>() + 2 pages, so the fetch cursor never laps the compute cursor
+  static constexpr int kPages = MM ? 6 : 12;
+  using Page = PageT<MM ? 32 : kMaxEntries>;
   // X of each accumulator (bf16 MMA operand, 128 rows x 64 keys, 128-byte swizzle).  Each buffer
   // starts 128 bytes further into the swizzle pattern than the one before, so the same row and
   // chunk of the receivers' buffers fall in different banks.  The tensor core applies the swizzle
   // to absolute shared-memory addresses (as TMA does): row r of buffer a has phase (r + a) % 8 and
   // the descriptor is the plain one (measured: a base offset of a in the descriptor reads wrong data).
   __nv_bfloat16 x[kAcc][128 * 64 + 64];
-  char x_align[1024 - kAcc * 128 % 1024];  // V on a 1024-byte boundary
+  // puts V on a 1024-byte boundary; the tensor-core mixing stores the zero rows of its products here
+  uint4 xscratch[(1024 - kAcc * 128 % 1024) / 16];
   __nv_bfloat16 v[kAcc][64 * 128];
-  uint4 ring[queue_of<F8>()][2][F8 ? kPieces8 : kPieces][kMixThreads];  // [pair slot][entry][piece][mixer thread]
-  uint4 xpad[8][32];  // tensor-core mixing: a 512-byte scratch per mixer warp for the zero rows of its products
+  // CUDA-core mixing: [pair slot][entry][piece][mixer thread]; tensor-core mixing: [warp][slot][2 KB]
+  uint4 ring[MM ? 8 * kMmSlots * 128 : queue_of<F8>() * 2 * (F8 ? kPieces8 : kPieces) * kMixThreads];
   Page page[kPages];
   uint64_t plan_full[kPages], plan_empty[kPages];
   uint64_t x_full, x_empty, v_full, v_empty, o_full, o_empty, mma_done;
@@ -123,9 +130,12 @@ struct SmemT {
   int abort;
 };
 
-static_assert(offsetof(SmemT<false>, v) % 1024 == 0 && offsetof(SmemT<true>, v) % 1024 == 0,
+using SmemBf16 = SmemT<false, false>;
+using SmemFp8 = SmemT<true, false>;
+using SmemMm = SmemT<false, true>;
+static_assert(offsetof(SmemBf16, v) % 1024 == 0 && offsetof(SmemFp8, v) % 1024 == 0 && offsetof(SmemMm, v) % 1024 == 0,
               "V is a 128-byte-swizzled TMA destination");
-static_assert(sizeof(SmemT<false>) + 1024 <= 232448 && sizeof(SmemT<true>) + 1024 <= 232448,
+static_assert(sizeof(SmemBf16) + 1024 <= 232448 && sizeof(SmemFp8) + 1024 <= 232448 && sizeof(SmemMm) + 1024 <= 232448,
               "shared memory of one CTA (plus alignment slack) must fit the 227 KB opt-in limit");
 
 struct Unit {
@@ -231,8 +241,10 @@ struct RowCursor {
 // ------------------------------------------------------------------------------------------------
 // Planner warp: pages (one per sub-step, plus a marker after every unit and one at the end).  It
 // waits only for page slots, never for the tensor core.
-template <int G, bool F8>
-__device__ void planner(SmemT<F8>& s, const Params& p) {
+template <int G, bool F8, bool MM>
+__device__ void planner(SmemT<F8, MM>& s, const Params& p) {
+  using Page = typename SmemT<F8, MM>::Page;
+  constexpr int kPages = SmemT<F8, MM>::kPages;
   const int lane = threadIdx.x & 31;
   uint32_t np = 0;    // pages written
   const int nparts = p.B / 64;
@@ -475,8 +487,8 @@ __device__ void issue_v(S& s, const Params& p, const CUtensorMap* tmap_v, const 
 
 // MMA warp: per sub-step, X (from the mixers) x V (loaded here one sub-step ahead) into the unit's
 // accumulators; the next V load is issued once these MMAs have read the buffer.
-template <int G, bool F8>
-__device__ void mma_issuer(SmemT<F8>& s, const Params& p, const CUtensorMap* tmap_v) {
+template <int G, bool F8, bool MM>
+__device__ void mma_issuer(SmemT<F8, MM>& s, const Params& p, const CUtensorMap* tmap_v) {
   const int lane = threadIdx.x & 31;
   const uint32_t idesc = idesc_bf16_f32(128, 128, false, true);
   const uint32_t tbase = s.tmem_base;
@@ -647,7 +659,9 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 // MM: mix on the tensor core with register operands (bf16 maps, block 128, at most 32 sender heads,
 // 4 receiver heads of one request group); otherwise in fp32 / half FMAs on the CUDA cores.
 template <int G, bool F8, bool MM>
-__device__ void mixers(SmemT<F8>& s, const Params& p) {
+__device__ void mixers(SmemT<F8, MM>& s, const Params& p) {
+  using Page = typename SmemT<F8, MM>::Page;
+  constexpr int kPages = SmemT<F8, MM>::kPages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int half = p.B == 64 ? (warp / (kMixWarps / 2)) : 0;  // 64-key blocks: which of the unit's two query blocks
   const uint32_t rowb = (uint32_t)(kRowsW * warp + (lane >> 3));
@@ -706,7 +720,7 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
   // copy the next pair's pieces into ring slot `slot` (one cp.async group per pair, empty when
   // there is nothing to copy, so group counts stay aligned with pairs); the move to the
   // following page is taken lazily, at the next call
-  const uint32_t ring0 = smem_u32(&s.ring[0][0][0][threadIdx.x]);
+  const uint32_t ring0 = smem_u32(&s.ring[threadIdx.x]);
   constexpr int kPc = F8 ? kPieces8 : kPieces;
   constexpr uint32_t kPiece = kMixThreads * 16u, kEntry = kPc * kPiece, kSlot = 2u * kEntry;
   constexpr int kQueue = queue_of<F8>();
@@ -919,11 +933,11 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
     // sender heads, copied by the warp into a private 2 KB slot of a 4-deep ring, so the warp waits
     // on its own copies only.  Head e's row sits at e * 128 with the map's physical chunk q at
     // q ^ (e % 8), so the eight rows of each transposed load hit eight different bank groups.
-    constexpr uint32_t kD = 4, kRows = 16;
+    constexpr uint32_t kD = kMmSlots, kRows = 16;
     constexpr uint32_t kHold = 2;  // rows computed before the wait for X (measured: 2 beats 3)
-    static_assert(sizeof(s.ring) == 8 * kD * 2048, "8 warps x kD slots of 2 KB");
+    static_assert(!MM || sizeof(s.ring) == 8 * kD * 2048, "8 warps x kD slots of 2 KB");
     static_assert(!MM || G == 4, "the first four rows of the product are the receiver heads");
-    char* wring_g = reinterpret_cast<char*>(&s.ring[0][0][0][0]) + (uint32_t)warp * (kD * 2048u);
+    char* wring_g = reinterpret_cast<char*>(&s.ring[0]) + (uint32_t)warp * (kD * 2048u);
     const uint32_t wring = smem_u32(wring_g);
     for (uint32_t off = (uint32_t)lane * 16u; off < kD * 2048u; off += 512u)
       *reinterpret_cast<uint4*>(wring_g + off) = make_uint4(0u, 0u, 0u, 0u);  // unlisted heads: weight 0, finite values
@@ -940,7 +954,7 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
     // go to scratch line r - 4 of this warp at the phases (R + r) % 8 the receivers leave free, so
     // the eight rows of each matrix fall in eight different bank groups
     const bool st_real = q < 4u;
-    const uint32_t st_base = st_real ? smem_u32(&s.x[q & 3u][0]) : smem_u32(&s.xpad[warp][0]) + (q - 4u) * 128u;
+    const uint32_t st_base = st_real ? smem_u32(&s.x[q & 3u][0]) : smem_u32(&s.xscratch[0]) + (q - 4u) * 128u;
     const uint32_t st_rowmask = st_real ? 0xffffffffu : 0u;
     const uint32_t st_u0 = lh << 4;
     auto store_row = [&](uint32_t row, const uint32_t (&w)[8]) {
@@ -1038,7 +1052,8 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
       cp_async_commit();
     };
     // one k-step of a row: wait for its slot, load it as B fragments, multiply, refill the slot with
-    // the step kD ahead: (row + kD / NKT, KT) of this page, or (TAIL) the next page's first steps
+    // the step kD ahead: (row + (KT + kD) / NKT, (KT + kD) % NKT) of this page, or (TAIL) the
+    // cursor's next step
     auto kstep = [&](uint32_t row, float (&acc)[8][4], auto KT, auto NKT, auto TAIL) {
       cp_async_wait<kD - 1>();  // this lane's copies of the oldest step have landed
       __syncwarp();             // ... and every other lane's
@@ -1058,9 +1073,10 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
       if constexpr (decltype(TAIL)::value) {
         if (!fetch_step(slot)) good = false;
       } else {
-        fetch_static(slot, row + kD / decltype(NKT)::value, KT);
+        constexpr int kN = decltype(NKT)::value, kAhead = decltype(KT)::value + (int)kD;
+        fetch_static(slot, row + (uint32_t)(kAhead / kN), Int<kAhead % kN>{});
       }
-      slot = (slot + 1u) & (kD - 1u);
+      slot = slot + 1u == kD ? 0u : slot + 1u;
     };
     // a whole row: its k-steps, then the receivers' X values packed to bf16
     auto row_x = [&](uint32_t row, uint32_t (&pk)[8], auto NKT, auto TAIL) {
@@ -1071,11 +1087,13 @@ __device__ void mixers(SmemT<F8>& s, const Params& p) {
       for (int nt = 0; nt < 8; ++nt) pk[nt] = pack_bf16x2(acc[nt][0], acc[nt][1]);
     };
     // the warp's 16 rows of one sub-step; rows 0..kHold are held until X is free.  On entry the fetch
-    // cursor has copied the page's first kD steps; the rest of the page is fetched statically and
-    // the last rows fetch the next page's first kD steps through the cursor.
+    // cursor has copied the page's first kD steps.  Rows before kTail fetch kD steps ahead within
+    // the page; the rest fetch through the cursor, which resumes at the first step they leave (the
+    // page's last steps, then the next page's first kD).
     auto sub_step = [&](auto NKT) -> bool {
-      constexpr uint32_t kTail = kRows - kD / decltype(NKT)::value;
-      f_s = f_steps;
+      constexpr uint32_t kN = decltype(NKT)::value;
+      constexpr uint32_t kTail = kRows - (kD + kN - 1) / kN;
+      f_s = kTail * kN + kD;
       uint32_t held[kHold + 1][8];
 #pragma unroll
       for (uint32_t r = 0; r <= kHold; ++r) row_x(r, held[r], NKT, Int<0>{});
@@ -1172,10 +1190,10 @@ template <int G, bool F8, bool MM>
 __global__ void __launch_bounds__(Roles<MM>::kThreadsK, 1) k_retrieve_tc(const __grid_constant__ CUtensorMap tmap_v, Params p) {
   constexpr int kMixWarps = Roles<MM>::kMix, kPlanWarp = Roles<MM>::kPlan, kMmaWarp = Roles<MM>::kMma;
   extern __shared__ unsigned char smem_raw[];
-  SmemT<F8>& s = *reinterpret_cast<SmemT<F8>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+  SmemT<F8, MM>& s = *reinterpret_cast<SmemT<F8, MM>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kPages; ++i) {
+    for (int i = 0; i < SmemT<F8, MM>::kPages; ++i) {
       mbar_init(&s.plan_full[i], 1);
       mbar_init(&s.plan_empty[i], kMixWarps);
     }
@@ -1199,9 +1217,9 @@ __global__ void __launch_bounds__(Roles<MM>::kThreadsK, 1) k_retrieve_tc(const _
   if (warp < kMixWarps)
     mixers<G, F8, MM>(s, p);
   else if (warp == kPlanWarp)
-    planner<G, F8>(s, p);
+    planner<G, F8, MM>(s, p);
   else
-    mma_issuer<G, F8>(s, p, &tmap_v);
+    mma_issuer<G, F8, MM>(s, p, &tmap_v);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1210,7 +1228,7 @@ __global__ void __launch_bounds__(Roles<MM>::kThreadsK, 1) k_retrieve_tc(const _
 
 template <int G, bool F8, bool MM = false>
 cudaError_t launch_g(const RetrieveArgs& a, const Params& p, const CUtensorMap& tm, int grid, cudaStream_t st) {
-  const size_t smem = sizeof(SmemT<F8>) + 1024;
+  const size_t smem = sizeof(SmemT<F8, MM>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_retrieve_tc<G, F8, MM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps(kKRetrieveTc, st);
