@@ -7,6 +7,9 @@ Tolerances (stated once, used by every test):
   * block masses: |M_gpu - M_oracle| <= MASS_ATOL (fp32 accumulation of fp32 probabilities);
   * stored probabilities: bf16 |P - A| <= 2^-8 |A| + 1e-6; fp32 |P - A| <= 3e-5 |A| + 1e-9;
   * outputs: max |O_gpu - O_oracle(GPU kept sets)| <= OUT_TOL[dtype] * max |V| (2e-2 bf16, 1e-4 fp32).
+    For bf16 the path rounds the map values, the mixing weights (tensor-core mixing), X and O to bf16,
+    each at most 2^-9 relative on non-negative terms of a row that sums to at most 1, so the error is
+    at most 4 * 2^-9 max |V| < 8e-3 max |V|, inside the stated 2e-2.
   * fp8 (e4m3) maps: stored values |P - A| <= 2^-4 |A| + 3e-6 (half an e4m3 step relative, plus the
     subnormal step of a piece whose scale is at most 1/448); outputs within 7e-2 max |V|: each
     translated value is off by at most 2^-4 of itself, plus bf16 and half-precision rounding (< 2^-8)
