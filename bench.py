@@ -785,6 +785,7 @@ def main():
     # Every step copies its inputs from pinned host memory and reads its result back inside the
     # timed region.  Double-buffered: step k + 1's inputs go up on a copy stream and step k - 1's
     # output comes down on another while step k computes; the compute itself stays on one stream.
+    # Q and K go up first: the compression needs only them, and the retrieval waits for V and W.
     e2e = None
     if not args.no_e2e:
         h2d = sum(host[k].numel() * host[k].element_size() for k in host)
@@ -793,7 +794,7 @@ def main():
         Ohs = [torch.empty(O.shape, dtype=bf).pin_memory() for _ in range(2)]
         d2h = Ohs[0].numel() * Ohs[0].element_size()
         s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-        ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("in", "done", "out")}
+        ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("qk", "vw", "done", "out")}
 
         def e2e_steps(n):
             for k in range(n):
@@ -801,13 +802,17 @@ def main():
                 with torch.cuda.stream(s_in):
                     if k >= 2:
                         s_in.wait_event(ev["done"][b])  # step k - 2 has finished with this buffer
-                    for name in ("Q", "K", "V", "W"):
+                    for name in ("Q", "K"):
                         d[name].copy_(host[name], non_blocking=True)
-                    ev["in"][b].record(s_in)
-                stream.wait_event(ev["in"][b])
+                    ev["qk"][b].record(s_in)
+                    for name in ("V", "W"):
+                        d[name].copy_(host[name], non_blocking=True)
+                    ev["vw"][b].record(s_in)
+                stream.wait_event(ev["qk"][b])
                 if k >= 2:
                     stream.wait_event(ev["out"][b])  # step k - 2's output has been read back
                 mr.compress(d["Q"], d["K"], p, spec.block, bias=bias, scale=spec.scale, out=m, ws=ws_c, stream=stream)
+                stream.wait_event(ev["vw"][b])
                 mr.retrieve(m, d["W"], d["V"], out=d["O"], ws=ws_r, stream=stream)
                 ev["done"][b].record(stream)
                 with torch.cuda.stream(s_out):
@@ -833,7 +838,8 @@ def main():
         ems = max_over_ranks(ems, dist, "cuda")
         e2e = {"value": job_tokens_per_s(world, spec.L, ems), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": ems,
-               "pipeline": "inputs of step k+1 and output of step k-1 copied while step k computes"}
+               "pipeline": ("inputs of step k+1 and output of step k-1 copied while step k computes; "
+                            "a step's compression starts once its Q and K are up")}
         del dev_bufs
 
     # ---- what the receiver would otherwise run: dense causal attention of its 64 heads ----
