@@ -1183,8 +1183,13 @@ __device__ void mixers(SmemT<F8, MM>& s, const Params& p) {
 template <bool MM>
 struct Roles {
   static constexpr int kMix = MM ? 8 : kMixWarps;
-  static constexpr int kPlan = kMix, kMma = kMix + 1, kThreadsK = (kMix + 2) * 32;
+  static constexpr int kPlan = kMix, kMma = kMix + 1;
+  // tensor-core mixing: two idle warps complete a third warpgroup with the planner and the MMA
+  // warp, which gives up registers (setmaxnreg) to the mixers' two warpgroups
+  static constexpr int kThreadsK = MM ? 384 : (kMix + 2) * 32;
 };
+constexpr int kMmLaunchRegs = 168, kMmRegsControl = 104, kMmRegsMix = 200;
+static_assert(kMmRegsControl + 2 * kMmRegsMix == 3 * kMmLaunchRegs, "register split of the tensor-core mixing launch");
 
 template <int G, bool F8, bool MM>
 __global__ void __launch_bounds__(Roles<MM>::kThreadsK, 1) k_retrieve_tc(const __grid_constant__ CUtensorMap tmap_v, Params p) {
@@ -1214,12 +1219,27 @@ __global__ void __launch_bounds__(Roles<MM>::kThreadsK, 1) k_retrieve_tc(const _
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp < kMixWarps)
-    mixers<G, F8, MM>(s, p);
-  else if (warp == kPlanWarp)
-    planner<G, F8, MM>(s, p);
-  else
-    mma_issuer<G, F8, MM>(s, p, &tmap_v);
+  if constexpr (MM) {
+    // every warp of the control warpgroup gives its registers back before any role starts, so
+    // the mixers' increase never waits on a role
+    if (warp < kMixWarps) {
+      regs_inc<kMmRegsMix>();
+      mixers<G, F8, MM>(s, p);
+    } else {
+      regs_dec<kMmRegsControl>();
+      if (warp == kPlanWarp)
+        planner<G, F8, MM>(s, p);
+      else if (warp == kMmaWarp)
+        mma_issuer<G, F8, MM>(s, p, &tmap_v);
+    }
+  } else {
+    if (warp < kMixWarps)
+      mixers<G, F8, MM>(s, p);
+    else if (warp == kPlanWarp)
+      planner<G, F8, MM>(s, p);
+    else
+      mma_issuer<G, F8, MM>(s, p, &tmap_v);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1229,7 +1249,15 @@ __global__ void __launch_bounds__(Roles<MM>::kThreadsK, 1) k_retrieve_tc(const _
 template <int G, bool F8, bool MM = false>
 cudaError_t launch_g(const RetrieveArgs& a, const Params& p, const CUtensorMap& tm, int grid, cudaStream_t st) {
   const size_t smem = sizeof(SmemT<F8, MM>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(k_retrieve_tc<G, F8, MM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e;
+  if (MM) {
+    // the register split assumes the launch allocation it was sized for
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, k_retrieve_tc<G, F8, MM>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kMmLaunchRegs) return cudaErrorInvalidConfiguration;
+  }
+  e = cudaFuncSetAttribute(k_retrieve_tc<G, F8, MM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps(kKRetrieveTc, st);
   k_retrieve_tc<G, F8, MM><<<grid, Roles<MM>::kThreadsK, smem, st>>>(tm, p);
