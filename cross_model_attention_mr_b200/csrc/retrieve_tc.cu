@@ -49,7 +49,7 @@ constexpr int kPieces = 128 * 8 / kMixThreads;           // 16-byte pieces per t
 template <bool F8>
 __host__ __device__ constexpr int queue_of() { return F8 ? 4 : 2; }
 constexpr int kMaxEntries = 64; // sender heads
-constexpr uint32_t kMmSlots = 5;  // tensor-core mixing: 2 KB ring slots per mixer warp
+constexpr uint32_t kMmSlots = 6;  // tensor-core mixing: 2 KB ring slots per mixer warp
 constexpr int kPaceSlack = 4;   // pages a CTA may run ahead of the slowest CTA of its group
 constexpr uint64_t kPaceNs = 100000ull;  // longest hold per page
 constexpr int kAcc = 4;
@@ -84,17 +84,24 @@ struct Params {
 
 // One listed panel: the tile of each of the unit's two query blocks (kNone: not kept, or never
 // stored because the map overflowed) and the unit's mixing weights for the panel's sender head.
-struct Entry {
+template <bool SC>
+struct EntryT {
   uint32_t t[2];
   uint32_t sc[2];  // fp8 maps: the scale of each 32-row group q of the unit in this panel, as bf16
                    // (group q in half q % 2 of word q / 2); unused for bf16 maps
   float w[kAcc];
 };
+template <>
+struct EntryT<false> {  // the tensor-core mixing's entries (bf16 maps): no scales
+  uint32_t t[2];
+  float w[kAcc];
+};
+using Entry = EntryT<true>;
 // One sub-step (n >= 1 entries, panel h of the key block) or a marker (n == 0).
-template <int E>
+template <int E, bool SC>
 struct PageT {
   uint32_t n, h, flags, pad;
-  Entry e[E];
+  EntryT<SC> e[E];
 };
 constexpr uint32_t kUnitEnd = 1u, kEmptyUnit = 2u, kEnd = 4u;
 
@@ -105,24 +112,41 @@ constexpr int kPieces8 = 1;
 constexpr float kF8Pre = 16384.f;
 constexpr float kF8Decode = 256.f;  // the integer decode yields value * 2^-8
 
-// MM: the tensor-core mixing (bf16 maps, at most 32 sender heads), with its own ring and a smaller
-// page ring (its fetch cursor is at most one page ahead of the compute cursor).
+// Shared memory of the CUDA-core mixing (MM = false); the tensor-core mixing has its own layout below.
 template <bool F8, bool MM>
 struct SmemT {
-  // CUDA-core mixing: > 2 * queue_of<true>() + 2 pages, so the fetch cursor never laps the compute cursor
-  static constexpr int kPages = MM ? 6 : 12;
-  using Page = PageT<MM ? 32 : kMaxEntries>;
+  // > 2 * queue_of<true>() + 2 pages, so the fetch cursor never laps the compute cursor
+  static constexpr int kPages = 12;
+  using Page = PageT<kMaxEntries, true>;
   // X of each accumulator (bf16 MMA operand, 128 rows x 64 keys, 128-byte swizzle).  Each buffer
   // starts 128 bytes further into the swizzle pattern than the one before, so the same row and
   // chunk of the receivers' buffers fall in different banks.  The tensor core applies the swizzle
   // to absolute shared-memory addresses (as TMA does): row r of buffer a has phase (r + a) % 8 and
   // the descriptor is the plain one (measured: a base offset of a in the descriptor reads wrong data).
   __nv_bfloat16 x[kAcc][128 * 64 + 64];
-  // puts V on a 1024-byte boundary; the tensor-core mixing stores the zero rows of its products here
-  uint4 xscratch[(1024 - kAcc * 128 % 1024) / 16];
+  char x_align[1024 - kAcc * 128 % 1024];  // V on a 1024-byte boundary
   __nv_bfloat16 v[kAcc][64 * 128];
-  // CUDA-core mixing: [pair slot][entry][piece][mixer thread]; tensor-core mixing: [warp][slot][2 KB]
-  uint4 ring[MM ? 8 * kMmSlots * 128 : queue_of<F8>() * 2 * (F8 ? kPieces8 : kPieces) * kMixThreads];
+  uint4 ring[queue_of<F8>() * 2 * (F8 ? kPieces8 : kPieces) * kMixThreads];  // [pair slot][entry][piece][mixer thread]
+  Page page[kPages];
+  uint64_t plan_full[kPages], plan_empty[kPages];
+  uint64_t x_full, x_empty, v_full, v_empty, o_full, o_empty, mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+// The tensor-core mixing (bf16 maps, at most 32 sender heads) fills the opt-in limit: V first (on
+// the 1024-byte boundary its swizzle needs), then the staggered X buffers, whose 128-byte gaps take
+// the zero rows of the matrix stores, a ring of kMmSlots 2 KB slots per mixer warp, and three pages
+// of 32 entries.  Three pages suffice: the fetch cursor is at most one page (kMmSlots steps < 16)
+// and one unit-end marker ahead of the compute cursor, and at 128-key blocks no unit is empty, so
+// markers never follow one another.  The launch adds no alignment slack; the kernel checks that
+// its dynamic shared memory starts on a 1024-byte boundary.
+template <bool F8>
+struct SmemT<F8, true> {
+  static constexpr int kPages = 3;
+  using Page = PageT<32, false>;
+  __nv_bfloat16 v[kAcc][64 * 128];
+  __nv_bfloat16 x[kAcc][128 * 64 + 64];
+  uint4 ring[8 * kMmSlots * 128];  // [mixer warp][slot][2 KB]
   Page page[kPages];
   uint64_t plan_full[kPages], plan_empty[kPages];
   uint64_t x_full, x_empty, v_full, v_empty, o_full, o_empty, mma_done;
@@ -133,10 +157,12 @@ struct SmemT {
 using SmemBf16 = SmemT<false, false>;
 using SmemFp8 = SmemT<true, false>;
 using SmemMm = SmemT<false, true>;
-static_assert(offsetof(SmemBf16, v) % 1024 == 0 && offsetof(SmemFp8, v) % 1024 == 0 && offsetof(SmemMm, v) % 1024 == 0,
-              "V is a 128-byte-swizzled TMA destination");
-static_assert(sizeof(SmemBf16) + 1024 <= 232448 && sizeof(SmemFp8) + 1024 <= 232448 && sizeof(SmemMm) + 1024 <= 232448,
+static_assert(offsetof(SmemBf16, v) % 1024 == 0 && offsetof(SmemFp8, v) % 1024 == 0 && offsetof(SmemMm, v) == 0 &&
+                  offsetof(SmemMm, x) % 1024 == 0,
+              "V and X are 128-byte-swizzled operands");
+static_assert(sizeof(SmemBf16) + 1024 <= 232448 && sizeof(SmemFp8) + 1024 <= 232448,
               "shared memory of one CTA (plus alignment slack) must fit the 227 KB opt-in limit");
+static_assert(sizeof(SmemMm) <= 232448, "the tensor-core mixing's shared memory must fit the 227 KB opt-in limit");
 
 struct Unit {
   int rb, hg, rg, I0, I1, Jmax;
@@ -343,7 +369,7 @@ __device__ void planner(SmemT<F8, MM>& s, const Params& p) {
             const int sh = lane + 32 * hs;
             if (!((uni >> sh) & 1ull)) continue;
             const int rank = __popcll((long long)(uni & ((1ull << sh) - 1ull)));
-            Entry& e = pg->e[rank];
+            auto& e = pg->e[rank];
 #pragma unroll
             for (int pt = 0; pt < 2; ++pt) {
               uint32_t t = kNone;
@@ -367,7 +393,7 @@ __device__ void planner(SmemT<F8, MM>& s, const Params& p) {
             }
 #pragma unroll
             for (int g = 0; g < kAcc; ++g) e.w[g] = wv[hs][g];
-            if (F8) {
+            if constexpr (F8) {
               // the scales of the unit's four 32-row groups in panel h (rows 32 q .. of query block
               // I0 at block 128; two groups of I0 and two of I1 at block 64), rounded to bf16: the
               // relative error 2^-9 is small beside the e4m3 step of the values they scale
@@ -769,7 +795,7 @@ __device__ void mixers(SmemT<F8, MM>& s, const Params& p) {
     }
 
   // fp8 entry: acch[g] += (W[r_g, s] * scale * 2^14) * (the thread's 16 e4m3 values)
-  auto mix_entry8 = [&](const Entry& E, uint32_t data) {
+  auto mix_entry8 = [&](const auto& E, uint32_t data) {
     const uint32_t scw = E.sc[rowb8 >> 6];
     const float sc = __uint_as_float((rowb8 & 32u) ? (scw & 0xffff0000u) : (scw << 16)) * (kF8Pre * kF8Decode);
     __half2 w2[G];
@@ -789,7 +815,7 @@ __device__ void mixers(SmemT<F8, MM>& s, const Params& p) {
   };
 
   // one entry: acc[g] += W[r_g, s] * (this thread's 16 values of the sender head's panel)
-  auto mix_entry = [&](const Entry& E, uint32_t data) {
+  auto mix_entry = [&](const auto& E, uint32_t data) {
     const float4 wf = *reinterpret_cast<const float4*>(&E.w[0]);
     const float w[4] = {wf.x, wf.y, wf.z, wf.w};
     float2 w2[G];
@@ -951,10 +977,10 @@ __device__ void mixers(SmemT<F8, MM>& s, const Params& p) {
     const uint32_t ld_row = (8u * (lh & 1u) + q) * 128u, ld_z = (lh >> 1) ^ q;
     // matrix stores of a finished row: lane 8 m + r gives row r of n-tile 4 k + m.  Rows r < 4 are
     // the receiver heads' X rows (swizzle phase (R + r) % 8); rows 4..7 of the product are zero and
-    // go to scratch line r - 4 of this warp at the phases (R + r) % 8 the receivers leave free, so
+    // go to the 128-byte gap after X buffer r - 4, at the phases (R + r) % 8 the receivers leave free, so
     // the eight rows of each matrix fall in eight different bank groups
     const bool st_real = q < 4u;
-    const uint32_t st_base = st_real ? smem_u32(&s.x[q & 3u][0]) : smem_u32(&s.xscratch[0]) + (q - 4u) * 128u;
+    const uint32_t st_base = smem_u32(st_real ? &s.x[q & 3u][0] : &s.x[q & 3u][128 * 64]);  // gap after buffer r - 4
     const uint32_t st_rowmask = st_real ? 0xffffffffu : 0u;
     const uint32_t st_u0 = lh << 4;
     auto store_row = [&](uint32_t row, const uint32_t (&w)[8]) {
@@ -1150,9 +1176,9 @@ __device__ void mixers(SmemT<F8, MM>& s, const Params& p) {
     const uint32_t data = ring0 + slot * kSlot;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      const Entry& E = cpg->e[2 * ec + j];
+      const auto& E = cpg->e[2 * ec + j];
       if (E.t[half] != kNone) {
-        if (F8)
+        if constexpr (F8)
           mix_entry8(E, data + j * kEntry);
         else
           mix_entry(E, data + j * kEntry);
@@ -1195,7 +1221,15 @@ template <int G, bool F8, bool MM>
 __global__ void __launch_bounds__(Roles<MM>::kThreadsK, 1) k_retrieve_tc(const __grid_constant__ CUtensorMap tmap_v, Params p) {
   constexpr int kMixWarps = Roles<MM>::kMix, kPlanWarp = Roles<MM>::kPlan, kMmaWarp = Roles<MM>::kMma;
   extern __shared__ unsigned char smem_raw[];
-  SmemT<F8, MM>& s = *reinterpret_cast<SmemT<F8, MM>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  if constexpr (MM) {
+    // no slack to align in this layout: the dynamic shared memory must start on a 1024-byte boundary
+    if (pad != 0) {
+      if (threadIdx.x == 0) set_status(p.ws, MR_ERR_DEVICE_CHECK, 9u);
+      return;
+    }
+  }
+  SmemT<F8, MM>& s = *reinterpret_cast<SmemT<F8, MM>*>(smem_raw + pad);
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int i = 0; i < SmemT<F8, MM>::kPages; ++i) {
@@ -1248,7 +1282,7 @@ __global__ void __launch_bounds__(Roles<MM>::kThreadsK, 1) k_retrieve_tc(const _
 
 template <int G, bool F8, bool MM = false>
 cudaError_t launch_g(const RetrieveArgs& a, const Params& p, const CUtensorMap& tm, int grid, cudaStream_t st) {
-  const size_t smem = sizeof(SmemT<F8, MM>) + 1024;
+  const size_t smem = sizeof(SmemT<F8, MM>) + (MM ? 0 : 1024);
   cudaError_t e;
   if (MM) {
     // the register split assumes the launch allocation it was sized for

@@ -294,7 +294,9 @@ typedef struct {
  *           checks strided layouts before launch (MR_ERR_INVALID_ARG); with a device offset table,
  *           a request whose rows do not fit inside [0, v_elems) (or, on the tensor-core kernel,
  *           whose offset is not a multiple of d_v) reads zeros instead and records
- *           MR_ERR_DEVICE_CHECK in the status word.
+ *           MR_ERR_DEVICE_CHECK in the status word.  The tensor-core mixing kernel (bf16 maps of
+ *           128-key blocks, at most 32 sender heads) also records MR_ERR_DEVICE_CHECK, writing no
+ *           output, if the device places its dynamic shared memory off a 1024-byte boundary.
  *   O       output in dtype dt: element (q, r, i, c) at O + q * H_r * L * d_v + (r * L + i) * d_v + c
  *   opts    NULL or mr_retrieve_opts
  *   ws      workspace of at least mr_retrieve_workspace_bytes(map, H_r, d_v, n_req) bytes
