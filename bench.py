@@ -145,6 +145,12 @@ def algorithmic(spec, nnz: int, union_tiles: int, n_req: int = 1, suffixes=None,
     }
 
 
+def mean_work(per_layer):
+    """Layer mean of the algorithmic work dicts: numbers averaged, labels (the first layer's) kept."""
+    return {k: (sum(w[k] for w in per_layer) / len(per_layer) if isinstance(v, (int, float)) else v)
+            for k, v in per_layer[0].items()}
+
+
 def kernel_work(name: str, work: dict):
     """(bound, amount, unit) of a kernel's algorithmic work per launch, against the roof the method
     names for its stage: the tensor-core peak for the contractions (QK^T in compression; the head
@@ -495,7 +501,7 @@ def run_config_line(args, spec, n):
     tokens = config_tokens_per_step(spec, suffixes)
     n_req = spec.n_req if n == 5 else 1
     per_layer = [algorithmic(spec, nnz, un, n_req, suffixes) for nnz, un in maps]
-    work = {k: sum(w[k] for w in per_layer) / len(per_layer) for k in per_layer[0]}  # per launch, layer mean
+    work = mean_work(per_layer)  # per launch, layer mean
     pk, pk_src = peaks()
     dname, (dms, dcnt) = max(prof.items(), key=lambda kv: kv[1][0])
     roofline = roofline_of(dname, dms, dcnt, work, pk, pk_src)

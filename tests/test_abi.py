@@ -71,6 +71,26 @@ def test_bench_traffic_is_tied_to_its_workload_and_sources():
         assert bench.traffic_for(kernel, "L8192_32to64_d128_bf16_B128") is None
 
 
+def test_bench_work_of_the_config_lines():
+    """The --config lines average the per-layer algorithmic work and keep its labels (which
+    head-mixing path the retrieval takes) as they are."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    from cross_model_attention_mr_b200.workloads import config
+    c2, c4 = config(2), config(4)
+    assert bench.algorithmic(c2, 100, 50)["mix_path"] == "cuda_core"       # 64-key blocks
+    assert bench.algorithmic(c4, 100, 50)["mix_path"] == "tensor"          # bf16, 128-key blocks, 32 heads
+    assert bench.algorithmic(c4, 100, 50, fp8=True)["mix_path"] == "cuda_core"
+    assert bench.algorithmic(c4, 100, 50, n_req=4)["mix_path"] == "cuda_core"
+    layers = [bench.algorithmic(c2, nnz, un) for nnz, un in ((100, 50), (300, 70))]
+    m = bench.mean_work(layers)
+    assert m["mix_path"] == "cuda_core"
+    assert m["map_bytes"] == (layers[0]["map_bytes"] + layers[1]["map_bytes"]) / 2
+    assert m["compress_flops"] == layers[0]["compress_flops"]
+
+
 def test_status_strings(mr):
     for code in range(8):
         s = mr.LIB.mr_status_string(code)
