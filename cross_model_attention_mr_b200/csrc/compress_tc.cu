@@ -49,6 +49,7 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.0f;  // move the row reference only for a jump of more than 2^8
+constexpr float kRescaleSum = 256.0f;  // 2^kRescale
 
 struct Params {
   int H, L, B, nqb, nkw, n_rb, n_units;
@@ -276,54 +277,95 @@ __device__ void softmax_group(Smem& s, const Params& p, int w) {
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.s_empty[w]);
-      float mc;
-      if (!special) {
-        // only the key-block term can apply: a constant per 32 keys
-        mc = -INFINITY;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) mc = fmaxf(mc, fmaf(warp_max32(v[cc]), p.a, kbo[cc]));
-      } else {
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int j0 = j_tile + 32 * cc;
-          const float kb = kb_term(p.bias, h, j0);
-#pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            const int j = j0 + t;
-            v[cc][t] = (row_ok && j <= i) ? fmaf(v[cc][t], p.a, bias_with_kb(p.bias, i, j, kb) * kLog2e) : -INFINITY;
-          }
-        }
-        mc = fmaxf(fmaxf(warp_max32(v[0]), warp_max32(v[1])), fmaxf(warp_max32(v[2]), warp_max32(v[3])));
-      }
-      if (!row_ok) mc = -INFINITY;
-      const bool need = mc > c + kRescale;
-      if (__any_sync(0xffffffffu, need)) {
-        const float cn = need ? mc : c;
-        const float f = need ? ex2_approx(c - cn) : 1.f;  // c = -inf gives 0
-        for (int c0 = 0; c0 < used; c0 += 32) {
-          uint32_t xs[32];
-          tmem_ld32(tbase + lane_addr + xbase + c0, xs);
-          tmem_wait_ld();
-#pragma unroll
-          for (int t = 0; t < 32; ++t) xs[t] = __float_as_uint(__uint_as_float(xs[t]) * f);
-          tmem_st32(tbase + lane_addr + xbase + c0, xs);
-        }
-        tmem_wait_st();
-        c = cn;
-      }
       float sum[4] = {0.f, 0.f, 0.f, 0.f};
-      if (c != -INFINITY && row_ok) {
+      // Ordinary tiles once the rows have a reference: the exponentials first, against it.  Their
+      // sum bounds their largest term, so a row whose sum is at most 2^kRescale has no logit more
+      // than kRescale above the reference, the max pass's own test, and gets that path's results.
+      // Otherwise (rare once the reference settles; also an overflow) the max of the shifted
+      // values moves the reference of the rows past it, and the exponentials are taken again.
+      if (!special && __all_sync(0xffffffffu, c != -INFINITY || !row_ok)) {
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
-          if (!special) {
-            const float o = kbo[cc] - c;
+          const float o = kbo[cc] - c;
 #pragma unroll
-            for (int t = 0; t < 32; ++t) v[cc][t] = fmaf(v[cc][t], p.a, o);
-          } else {
-#pragma unroll
-            for (int t = 0; t < 32; ++t) v[cc][t] -= c;  // -inf stays -inf and gives 0
-          }
+          for (int t = 0; t < 32; ++t) v[cc][t] = fmaf(v[cc][t], p.a, o);
           sum[cc] = sum_ex2_32(v[cc]);
+        }
+        const bool big = row_ok && !(((sum[0] + sum[1]) + (sum[2] + sum[3])) <= kRescaleSum);
+        if (__any_sync(0xffffffffu, big)) {
+          const float m = fmaxf(fmaxf(warp_max32(v[0]), warp_max32(v[1])), fmaxf(warp_max32(v[2]), warp_max32(v[3])));
+          const bool need = row_ok && m > kRescale;
+          if (__any_sync(0xffffffffu, need)) {
+            const float d = need ? m : 0.f;
+            const float f = need ? ex2_approx(-d) : 1.f;
+            for (int c0 = 0; c0 < used; c0 += 32) {
+              uint32_t xs[32];
+              tmem_ld32(tbase + lane_addr + xbase + c0, xs);
+              tmem_wait_ld();
+#pragma unroll
+              for (int t = 0; t < 32; ++t) xs[t] = __float_as_uint(__uint_as_float(xs[t]) * f);
+              tmem_st32(tbase + lane_addr + xbase + c0, xs);
+            }
+            tmem_wait_st();
+            c += d;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+              for (int t = 0; t < 32; ++t) v[cc][t] -= d;
+              sum[cc] = sum_ex2_32(v[cc]);
+            }
+          }
+        }
+        if (!row_ok) sum[0] = sum[1] = sum[2] = sum[3] = 0.f;
+      } else {
+        float mc;
+        if (!special) {
+          // only the key-block term can apply: a constant per 32 keys
+          mc = -INFINITY;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) mc = fmaxf(mc, fmaf(warp_max32(v[cc]), p.a, kbo[cc]));
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            const int j0 = j_tile + 32 * cc;
+            const float kb = kb_term(p.bias, h, j0);
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+              const int j = j0 + t;
+              v[cc][t] = (row_ok && j <= i) ? fmaf(v[cc][t], p.a, bias_with_kb(p.bias, i, j, kb) * kLog2e) : -INFINITY;
+            }
+          }
+          mc = fmaxf(fmaxf(warp_max32(v[0]), warp_max32(v[1])), fmaxf(warp_max32(v[2]), warp_max32(v[3])));
+        }
+        if (!row_ok) mc = -INFINITY;
+        const bool need = mc > c + kRescale;
+        if (__any_sync(0xffffffffu, need)) {
+          const float cn = need ? mc : c;
+          const float f = need ? ex2_approx(c - cn) : 1.f;  // c = -inf gives 0
+          for (int c0 = 0; c0 < used; c0 += 32) {
+            uint32_t xs[32];
+            tmem_ld32(tbase + lane_addr + xbase + c0, xs);
+            tmem_wait_ld();
+#pragma unroll
+            for (int t = 0; t < 32; ++t) xs[t] = __float_as_uint(__uint_as_float(xs[t]) * f);
+            tmem_st32(tbase + lane_addr + xbase + c0, xs);
+          }
+          tmem_wait_st();
+          c = cn;
+        }
+        if (c != -INFINITY && row_ok) {
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            if (!special) {
+              const float o = kbo[cc] - c;
+#pragma unroll
+              for (int t = 0; t < 32; ++t) v[cc][t] = fmaf(v[cc][t], p.a, o);
+            } else {
+#pragma unroll
+              for (int t = 0; t < 32; ++t) v[cc][t] -= c;  // -inf stays -inf and gives 0
+            }
+            sum[cc] = sum_ex2_32(v[cc]);
+          }
         }
       }
       // block sums of this tile: one 128-key block, or two 64-key blocks

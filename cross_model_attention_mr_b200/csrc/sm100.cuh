@@ -241,7 +241,9 @@ __device__ __forceinline__ float ex2_approx(float x) {
 template <int Deg>
 __device__ __forceinline__ float ex2_poly(float x) {
   static_assert(Deg == 3 || Deg == 5, "degree 3 or 5");
-  const float xc = fmaxf(x, -127.f);
+  // arguments above 127 give 2^127 (finite, larger than any sum the callers accept) rather than a
+  // wrapped exponent field
+  const float xc = fminf(fmaxf(x, -127.f), 127.f);
   const float t = __fadd_rn(xc, 12582912.f);
   const float f = __fsub_rn(xc, __fsub_rn(t, 12582912.f));
   float p;
