@@ -202,9 +202,10 @@ __device__ __forceinline__ float warp_max32(const float (&v)[32]) {
 }
 
 // Sum of 2^x over 32 values with 8 independent partial sums.  The values kEmuMask names (bit k:
-// value 8 m + k) take the FMA-pipe exponential of degree 5, the rest the multi-function unit,
-// whose 16 results per clock per SM otherwise bound this kernel.
-constexpr uint32_t kEmuMask = 0x88;
+// value 8 m + k) take the FMA-pipe exponential of degree 5, the rest the multi-function unit.
+// None do: with the exponentials taken before the max (most tiles need no max pass), the kernel is
+// no longer bound by the multi-function unit, and moving 1 or 2 of every 8 measured slower.
+constexpr uint32_t kEmuMask = 0x00;
 __device__ __forceinline__ float ex2_mixed(float x, int t) {
   return ((kEmuMask >> (t & 7)) & 1) ? ex2_poly<5>(x) : ex2_approx(x);
 }
