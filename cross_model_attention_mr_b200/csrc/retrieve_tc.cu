@@ -9,12 +9,14 @@
 //   * planner warp: for every sender head that kept the key block (bitmask union) writes one
 //     entry (tile index, the unit's mixing weights W[r, s]) into a page of a shared-memory ring,
 //     one page per sub-step, and pulls the sub-step's map panels into L2 ahead of use;
-//   * 16 mixer warps: each thread copies its own 2 x 16 bytes of every listed panel from L2 into
-//     a private shared-memory ring, two panels (sender heads) per slot (cp.async, per-thread
-//     completion: no per-panel barrier), accumulates the head mixing in fp32 (pairs of columns
-//     per FFMA2), and at the end
-//     of a sub-step writes X_r as a bf16 MMA operand to shared memory; the translated map exists
-//     only there, never in global memory;
+//   * mixer warps copy the listed panels from L2 into private shared-memory rings (cp.async,
+//     per-thread completion: no per-panel barrier), mix the sender heads, and write X_r as a bf16
+//     MMA operand to shared memory; the translated map exists only there, never in global memory.
+//     bf16 maps of 128-key blocks with at most 32 sender heads and 4 receiver heads per CTA: 8
+//     warps mix on the tensor core, one unit row x 16 sender heads per mma.sync step with fp32
+//     register accumulators (Tensor Memory holds the Ã·V accumulators).  Otherwise: 16 warps,
+//     each thread mixing its own 2 x 16 bytes of every listed panel in fp32 (pairs of columns per
+//     FFMA2) or, for fp8 maps, in pre-scaled half precision;
 //   * MMA warp: loads the receivers' V rows for the next sub-step with TMA (128-byte swizzle)
 //     once the current MMAs have read the buffer, and issues tcgen05.mma X_r (128 x 64, K-major)
 //     x V (64 x 128, MN-major) into the fp32 accumulators;
@@ -36,10 +38,11 @@ namespace {
 
 using namespace sm100;
 
-// 16 mixer warps + planner + MMA warp.  Five warps then share one SM sub-partition, which caps a
-// thread at 96 registers: enough for 4 x 16 fp32 accumulators (2 pieces per thread) with the
-// paired FMA as a compiler builtin.  Measured against 8 mixer warps with 4 pieces each (168
-// registers): 4 mixer warps per sub-partition hide more latency, 5% faster at 32K tokens.
+// CUDA-core mixing: 16 mixer warps + planner + MMA warp.  Five warps then share one SM
+// sub-partition, which caps a thread at 96 registers: enough for 4 x 16 fp32 accumulators (2
+// pieces per thread) with the paired FMA as a compiler builtin.  Measured against 8 mixer warps
+// with 4 pieces each (168 registers): 4 mixer warps per sub-partition hide more latency, 5% faster
+// at 32K tokens.
 constexpr int kMixWarps = 16;  // CUDA-core mixing path (the tensor-core one runs 8, see Roles)
 constexpr int kMixThreads = kMixWarps * 32;
 constexpr int kRowsW = 128 / kMixWarps;                  // unit rows per mixer warp
@@ -956,7 +959,7 @@ __device__ void mixers(SmemT<F8, MM>& s, const Params& p) {
     // transposed matrix load), accumulated in fp32 registers: no Tensor Memory (all of it holds the
     // Ã·V accumulators) and no per-thread accumulator arrays.  8 mixer warps; warp w owns unit rows
     // 16 w .. 16 w + 15.  A step is one row and one k-step: the row's 128 bytes in each of 16
-    // sender heads, copied by the warp into a private 2 KB slot of a 4-deep ring, so the warp waits
+    // sender heads, copied by the warp into a private 2 KB slot of a kMmSlots-deep ring, so the warp waits
     // on its own copies only.  Head e's row sits at e * 128 with the map's physical chunk q at
     // q ^ (e % 8), so the eight rows of each transposed load hit eight different bank groups.
     constexpr uint32_t kD = kMmSlots, kRows = 16;
