@@ -140,8 +140,10 @@ struct SmemT {
 // the 1024-byte boundary its swizzle needs), then the staggered X buffers, whose 128-byte gaps take
 // the zero rows of the matrix stores, a ring of kMmSlots 2 KB slots per mixer warp, and three pages
 // of 32 entries.  Three pages suffice: the fetch cursor is at most one page (kMmSlots steps < 16)
-// and one unit-end marker ahead of the compute cursor, and at 128-key blocks no unit is empty, so
-// markers never follow one another.  The launch adds no alignment slack; the kernel checks that
+// and one unit-end marker ahead of the compute cursor, and at 128-key blocks no unit is empty
+// (every query row sees its own key, a logit no bias masks, so with p > 0 every head keeps a
+// block of every query block), so markers never follow one another (the final end marker follows
+// a unit-end marker, which is the one marker and page the cursor may pass).  The launch adds no alignment slack; the kernel checks that
 // its dynamic shared memory starts on a 1024-byte boundary.
 template <bool F8>
 struct SmemT<F8, true> {
