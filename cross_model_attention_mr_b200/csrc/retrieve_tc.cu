@@ -965,7 +965,9 @@ __device__ void mixers(SmemT<F8, MM>& s, const Params& p) {
     // on its own copies only.  Head e's row sits at e * 128 with the map's physical chunk q at
     // q ^ (e % 8), so the eight rows of each transposed load hit eight different bank groups.
     constexpr uint32_t kD = kMmSlots, kRows = 16;
-    constexpr uint32_t kHold = 2;  // rows computed before the wait for X (measured: 2 beats 3)
+    // rows 0..kHold are computed before the wait for X (measured at 32K tokens with 200 registers:
+    // kHold 0 54.0 ms, 1 54.9, 2 55.9, 3 58.9)
+    constexpr uint32_t kHold = 0;
     static_assert(!MM || sizeof(s.ring) == 8 * kD * 2048, "8 warps x kD slots of 2 KB");
     static_assert(!MM || G == 4, "the first four rows of the product are the receiver heads");
     char* wring_g = reinterpret_cast<char*>(&s.ring[0]) + (uint32_t)warp * (kD * 2048u);
