@@ -301,7 +301,10 @@ typedef struct {
  *   opts    NULL or mr_retrieve_opts
  *   ws      workspace of at least mr_retrieve_workspace_bytes(map, H_r, d_v, n_req) bytes
  * Supported: d_v in {64, 128}; H_r <= 256.  bf16 maps with d_v = 128, block 64 or 128 and
- * H_s <= 64 run on the tensor-core kernel; other shapes on the CUDA-core kernel.
+ * H_s <= 64 run on the tensor-core kernel; other shapes on the CUDA-core kernel.  Within the
+ * tensor-core kernel, bf16 maps of 128-key blocks with H_s <= 32 and n_req <= 1 mix the sender
+ * heads on the tensor core too (weights rounded to bf16, fp32 accumulation); other maps mix them
+ * on the CUDA cores (bf16 maps in fp32, fp8 maps in half precision).
  * Tiles a map could not store (capacity overflow at compression) contribute nothing and set
  * MR_ERR_CAPACITY in the status word.
  */
